@@ -1,0 +1,416 @@
+#!/usr/bin/env python
+"""Benchmark of the quantized fused-MoE experts hot path on B200.
+
+One step = one pass of the whole path over one layer of the workload, inputs resident
+in HBM: NF4 (or NF4 + double quant, or row-wise int8) quantization of gate_up and
+down from bf16, dequantization of both, and the routed experts forward
+(route -> gather -> gate_up GEMM + SiLU*up -> down GEMM + weighted slots -> combine).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload olmoe] [--impl ours|reference]
+
+`value` is expert-forward TFLOP/s (algorithmic 6*T*K*H*I per step over the forward's
+device time, all ranks' work over the max over ranks); the line also carries the
+forward tokens/s, quantize and dequantize GB/s, per-kernel times, the roofline of the
+dominant kernel, the CPU oracle as a baseline, an end-to-end number through the C ABI
+with host buffers, SM clocks sampled during the timed region, and the kernel count.
+`--impl reference` times the CPU oracle on a bounded sample of the same workload.
+Multi-GPU (torchrun): every rank runs its own replica of the workload (the forward
+does not shard: no collective on the data path); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "expert-forward TFLOP/s & tokens/s, quantize GB/s; % of roofline (1×B200)"
+L2_BYTES = 126 * 2**20
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default="olmoe")
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=15.0)
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.f = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.sel = str(device)
+
+    def start(self):
+        try:
+            self.f = tempfile.TemporaryFile(mode="w+")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.sel, f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait()
+        self.f.seek(0)
+        rows = [r.split(", ") for r in self.f.read().strip().splitlines() if r.count(",") >= 8]
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timings (bounded samples)
+# ---------------------------------------------------------------------------
+def oracle_sample(wl, inputs_cpu: dict, seconds: float):
+    """Times the oracle forward on a few tokens and the oracle quantizer on one expert.
+    Returns (forward_tflops, tokens_per_s, quantize_gbs, sample_description, threads)."""
+    import numpy as np
+    import oracle as O
+    from threadpoolctl import threadpool_info
+
+    def bits(t):
+        return t.contiguous().view(torch.uint16).numpy()
+
+    mode_q = {0: lambda w: O.quantize_nf4(w), 1: lambda w: O.quantize_nf4(w, True),
+              2: O.quantize_int8_rowwise}[wl.mode]
+    # quantize: one expert of gate_up
+    w1 = bits(inputs_cpu["gate_up"][0:1])
+    t0 = time.perf_counter()
+    pk = mode_q(w1)
+    tq = time.perf_counter() - t0
+    from bit_weight_quantization_moeq_b200.synth import quantize_bytes
+    q_gbs = quantize_bytes(wl.mode, 1, 2 * wl.I, wl.H) / tq / 1e9
+    # forward: the first two tokens, their experts quantized and dequantized up front
+    # (not timed), the fp64 forward on them repeated until the time budget is used
+    idx = inputs_cpu["top_k_index"].numpy().astype(np.int64)
+    toks = np.arange(min(2, wl.T))
+    gu = np.zeros((wl.E, 2 * wl.I, wl.H), np.float32)
+    dn = np.zeros((wl.E, wl.H, wl.I), np.float32)
+    for e in sorted({int(e) for e in idx[toks].reshape(-1)}):
+        gu[e] = O.dequantize(mode_q(bits(inputs_cpu["gate_up"][e:e + 1])))[0]
+        dn[e] = O.dequantize(mode_q(bits(inputs_cpu["down"][e:e + 1])))[0]
+    x = bits(inputs_cpu["hidden"])
+    wts = inputs_cpu["top_k_weights"].float().numpy()
+    elapsed, done, reps = 0.0, 0, 0
+    while elapsed < seconds or reps < 2:
+        t0 = time.perf_counter()
+        O.experts_forward(x, idx, wts, gu, dn, tokens=toks)
+        elapsed += time.perf_counter() - t0
+        done += len(toks)
+        reps += 1
+    flops = 6.0 * done * wl.K * wl.H * wl.I
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    desc = (f"oracle fp64 forward (numpy BLAS) on the first {len(toks)} of {wl.T} tokens, repeated {reps}x "
+            f"in {elapsed:.1f} s; oracle quantize of 1 of {wl.E} gate_up experts in {tq:.2f} s")
+    return flops / elapsed / 1e12, done / elapsed, q_gbs, desc, threads
+
+
+# ---------------------------------------------------------------------------
+# our path
+# ---------------------------------------------------------------------------
+def run_ours(args, wl, rank, world, dev):
+    import bit_weight_quantization_moeq_b200 as M
+    from bit_weight_quantization_moeq_b200 import synth
+
+    pk = peaks()
+    torch.cuda.set_device(dev)
+    inputs = synth.workload_inputs(wl, device=f"cuda:{dev}")
+    T, K, E, H, I = wl.T, wl.K, wl.E, wl.H, wl.I
+    mode = wl.mode
+    gu_p = M.PackedWeight.empty(mode, E, 2 * I, H, f"cuda:{dev}")
+    dn_p = M.PackedWeight.empty(mode, E, H, I, f"cuda:{dev}")
+    qws = torch.empty(max(M.moeq_quantize_workspace(mode, E, 2 * I, H), 16), dtype=torch.uint8, device=f"cuda:{dev}")
+    dq_gu = torch.empty((E, 2 * I, H), dtype=torch.bfloat16, device=f"cuda:{dev}")
+    dq_dn = torch.empty((E, H, I), dtype=torch.bfloat16, device=f"cuda:{dev}")
+    fws = torch.empty(M.moeq_forward_workspace(T, K, E, H, I), dtype=torch.uint8, device=f"cuda:{dev}")
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=f"cuda:{dev}")
+
+    def quantize(w, p):
+        if mode == 2:
+            M.moeq_quantize_int8_rowwise(w, out=p)
+        else:
+            M.moeq_quantize_nf4(w, double_quant=(mode == 1), out=p, ws=qws)
+
+    def step(ev, tev):
+        ev[0].record()
+        quantize(inputs["gate_up"], gu_p)
+        ev[1].record()
+        quantize(inputs["down"], dn_p)
+        ev[2].record()
+        M.moeq_dequantize(gu_p, out=dq_gu)
+        M.moeq_dequantize(dn_p, out=dq_dn)
+        ev[3].record()
+        M.moeq_set_trace_events(tev)
+        M.moeq_experts_forward(inputs["hidden"], inputs["top_k_index"], inputs["top_k_weights"], gu_p, dn_p,
+                               out=out, ws=fws)
+        M.moeq_set_trace_events(None)
+        ev[4].record()
+
+    def mk(n):
+        return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+    for _ in range(args.warmup):
+        step(mk(5), mk(6))
+    torch.cuda.synchronize()
+    evs = [mk(5) for _ in range(args.steps)]
+    tevs = [mk(6) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev)
+    clocks.start()
+    l0 = M.moeq_kernel_launches()
+    t_start, t_end = mk(2)
+    t_start.record()
+    for i in range(args.steps):
+        step(evs[i], tevs[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    launches = M.moeq_kernel_launches() - l0
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+
+    def el(a, b):
+        return a.elapsed_time(b)
+
+    total_ms = el(t_start, t_end)
+    comp = {
+        "quantize_gate_up": sum(el(e[0], e[1]) for e in evs),
+        "quantize_down": sum(el(e[1], e[2]) for e in evs),
+        "dequantize": sum(el(e[2], e[3]) for e in evs),
+        "forward": sum(el(e[3], e[4]) for e in evs),
+        "route": sum(el(t[0], t[1]) for t in tevs),
+        "gather": sum(el(t[1], t[2]) for t in tevs),
+        "gemm_gate_up": sum(el(t[2], t[3]) for t in tevs),
+        "gemm_down": sum(el(t[3], t[4]) for t in tevs),
+        "combine": sum(el(t[4], t[5]) for t in tevs),
+    }
+    vals = torch.tensor([total_ms] + list(comp.values()), dtype=torch.float64, device=f"cuda:{dev}")
+    if world > 1:
+        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(vals[0])
+    comp = {k: float(v) / args.steps for k, v in zip(comp.keys(), vals[1:].tolist())}
+
+    from bit_weight_quantization_moeq_b200.synth import forward_flops, quantize_bytes
+    S = T * K
+    flops = forward_flops(T, K, H, I)
+    q_bytes = quantize_bytes(mode, E, 2 * I, H) + quantize_bytes(mode, E, H, I)
+    n_elem = E * 3 * I * H
+    packed_bytes = gu_p.nbytes() + dn_p.nbytes()
+    dq_bytes = packed_bytes + 2 * n_elem
+    fwd_tflops = world * flops / (comp["forward"] * 1e-3) / 1e12
+    # distinct experts hit (for the forward's algorithmic bytes)
+    hit = torch.unique(inputs["top_k_index"]).numel()
+    fwd_bytes = packed_bytes * hit / E + 2 * T * H * 2 + S * 8
+
+    kernels = {
+        "quantize_gate_up": {"bound": "hbm", "ms": comp["quantize_gate_up"],
+                             "bytes": quantize_bytes(mode, E, 2 * I, H)},
+        "gemm_gate_up": {"bound": "tensor", "ms": comp["gemm_gate_up"], "flops": 4.0 * S * H * I},
+        "gemm_down": {"bound": "tensor", "ms": comp["gemm_down"], "flops": 2.0 * S * H * I},
+        "quantize_down": {"bound": "hbm", "ms": comp["quantize_down"], "bytes": quantize_bytes(mode, E, H, I)},
+    }
+    for k, v in kernels.items():
+        if v["bound"] == "hbm":
+            v["achieved"] = v["bytes"] / (v["ms"] * 1e-3) / 1e9
+            v["peak"], v["unit"] = pk["hbm_gbs"], "GB/s"
+        else:
+            v["achieved"] = v["flops"] / (v["ms"] * 1e-3) / 1e12
+            v["peak"], v["unit"] = pk["bf16_tflops"], "TFLOP/s"
+        v["frac"] = v["achieved"] / v["peak"]
+    dom = max(kernels, key=lambda k: kernels[k]["ms"])
+    dk = kernels[dom]
+    roofline = {"kernel": dom, "bound": dk["bound"], "achieved": round(dk["achieved"], 2), "peak": dk["peak"],
+                "unit": dk["unit"], "frac": round(dk["frac"], 4), "traffic": None,
+                "peak_source": pk["source"] + (" burst" if dk["bound"] == "tensor" else " copy")}
+
+    result = {
+        "metric": METRIC, "value": round(fwd_tflops, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02) bf16 weights, N(0,1) hidden, softmax top-k routing)",
+        "config": {"workload": wl.label, "E": E, "H": H, "I": I, "top_k": K, "tokens": T,
+                   "mode": ["nf4", "nf4+double-quant", "int8-rowwise"][mode],
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (bf16 weights %.0f MB > 126 MB L2), no flush" % (2 * n_elem / 1e6)},
+        "forward": {"tflops": round(fwd_tflops, 3),
+                    "tokens_per_s": round(world * T / (comp["forward"] * 1e-3), 1),
+                    "ms": round(comp["forward"], 4),
+                    "bytes_gbs": round(fwd_bytes / (comp["forward"] * 1e-3) / 1e9, 1),
+                    "roofline_frac": round(max(flops / (pk["bf16_tflops"] * 1e12), fwd_bytes / (pk["hbm_gbs"] * 1e9))
+                                           / (comp["forward"] * 1e-3), 4)},
+        "quantize": {"gbs": round(world * q_bytes / ((comp["quantize_gate_up"] + comp["quantize_down"]) * 1e-3) / 1e9, 1),
+                     "ms": round(comp["quantize_gate_up"] + comp["quantize_down"], 4),
+                     "frac_of_hbm": round(q_bytes / ((comp["quantize_gate_up"] + comp["quantize_down"]) * 1e-3) / 1e9
+                                          / pk["hbm_gbs"], 4)},
+        "dequantize": {"gbs": round(dq_bytes / (comp["dequantize"] * 1e-3) / 1e9, 1),
+                       "ms": round(comp["dequantize"], 4)},
+        "kernel_ms": {k: round(v, 4) for k, v in comp.items()},
+        "kernels": {k: {"ms": round(v["ms"], 4), "achieved": round(v["achieved"], 2), "unit": v["unit"],
+                        "frac": round(v["frac"], 4)} for k, v in kernels.items()},
+        "roofline": roofline,
+        "clocks": clk,
+        "gpu_launches": int(launches),
+    }
+    return result, inputs
+
+
+def run_e2e(wl, dev, steps=3, warmup=1):
+    """Same forward metric through the C ABI with host buffers: every step copies its
+    inputs (bf16 weights, hidden, routing) from pinned host memory, quantizes,
+    dequantizes, runs the forward and reads the output back."""
+    import bit_weight_quantization_moeq_b200 as M
+    from bit_weight_quantization_moeq_b200 import synth
+    T, K, E, H, I, mode = wl.T, wl.K, wl.E, wl.H, wl.I, wl.mode
+    d = f"cuda:{dev}"
+    host = synth.workload_inputs(wl, device="cpu")
+    host = {k: v.pin_memory() for k, v in host.items()}
+    dv = {k: torch.empty_like(v, device=d) for k, v in host.items()}
+    gu_p = M.PackedWeight.empty(mode, E, 2 * I, H, d)
+    dn_p = M.PackedWeight.empty(mode, E, H, I, d)
+    qws = torch.empty(max(M.moeq_quantize_workspace(mode, E, 2 * I, H), 16), dtype=torch.uint8, device=d)
+    dq_gu = torch.empty((E, 2 * I, H), dtype=torch.bfloat16, device=d)
+    dq_dn = torch.empty((E, H, I), dtype=torch.bfloat16, device=d)
+    fws = torch.empty(M.moeq_forward_workspace(T, K, E, H, I), dtype=torch.uint8, device=d)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=d)
+    out_h = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+
+    def q(w, p):
+        if mode == 2:
+            M.moeq_quantize_int8_rowwise(w, out=p)
+        else:
+            M.moeq_quantize_nf4(w, double_quant=(mode == 1), out=p, ws=qws)
+
+    def step():
+        for k in host:
+            dv[k].copy_(host[k], non_blocking=True)
+        q(dv["gate_up"], gu_p)
+        q(dv["down"], dn_p)
+        M.moeq_dequantize(gu_p, out=dq_gu)
+        M.moeq_dequantize(dn_p, out=dq_dn)
+        M.moeq_experts_forward(dv["hidden"], dv["top_k_index"], dv["top_k_weights"], gu_p, dn_p, out=out, ws=fws)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    from bit_weight_quantization_moeq_b200.synth import forward_flops
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    return {"value": round(forward_flops(T, K, H, I) / (ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 3), "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(out_h.numel() * out_h.element_size()),
+            "note": "step includes the H2D upload of the bf16 weights being quantized on load"}, host
+
+
+def run_reference(args, wl):
+    """The CPU oracle on bounded samples of the same workload, one sample per step."""
+    from bit_weight_quantization_moeq_b200 import synth
+    inputs = synth.workload_inputs(wl, device="cpu")
+    per_step = max(2.0, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(wl, inputs, per_step / 4)
+    vals, descs = [], []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        tf, tps, qg, desc, thr = oracle_sample(wl, inputs, per_step)
+        vals.append(tf)
+        descs.append(desc)
+    wall = time.perf_counter() - t0
+    v = statistics.median(vals)
+    return {"metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(wall / args.steps * 1e3, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.label},
+            "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                             "sample": descs[-1]},
+            "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    from bit_weight_quantization_moeq_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, wl)), flush=True)
+        return
+    if world > 1:
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device(f"cuda:{local}"))
+    result, inputs = run_ours(args, wl, rank, world, local)
+    if rank == 0 and world == 1 and not args.no_e2e:
+        del inputs
+        torch.cuda.empty_cache()
+        result["e2e"], host = run_e2e(wl, local)
+        if not args.no_cpu_baseline:
+            tf, tps, qg, desc, thr = oracle_sample(wl, host, args.cpu_seconds)
+            result["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                                      "sample": desc, "tokens_per_s": round(tps, 3), "quantize_gbs": round(qg, 4)}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+if __name__ == "__main__":
+    main()

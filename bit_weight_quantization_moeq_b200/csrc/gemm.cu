@@ -1,0 +1,527 @@
+// Grouped expert GEMMs straight from packed NF4 / int8 weights (sm_100a, tcgen05 + TMEM).
+//
+// What is computed (bitsandbytes issue #1849, "Description": gate_up_proj [E, 2I, H],
+// down_proj [E, H, I], act = SiLU; the fused grouped NF4 GEMM described later in that
+// thread decodes NF4 inside the mainloop with fp32 accumulation and never materialises
+// a dequantized weight tensor):
+//   gate_up:  h[s, j] = silu(x_s . G_e[j]) * (x_s . U_e[j]),  G = rows [0, I), U = rows
+//             [I, 2I) of gate_up[e]  (gate is never inferred from the shape: unsloth-zoo
+//             issue #850 on the square OLMoE gate_up)
+//   down:     slot[p, i] = w_p * (h_s . D_e[i])   with p = perm[s] the (t, k) pair of s
+// over the expert-sorted rows s of each expert e.
+//
+// Tile = 128 weight rows (UMMA M, operand A) x up to 256 tokens (UMMA N, operand B) x
+// K in steps of 64 (one NF4 block, one 128-byte swizzle row).
+//   warps 0-3  epilogue: TMEM -> registers (tcgen05.ld), SiLU*up or weighted slot stores
+//   warps 4-7  dequant: packed codes (TMA'd into SMEM) -> bf16 A tile in the UMMA
+//              K-major 128B-swizzled layout, one weight row per thread
+//   warp 8     producer: TMA of the token tile (B, 128B swizzle) and of the code tiles
+//   warp 9     TMEM allocation and the single-thread tcgen05.mma issue
+// Accumulators are double-buffered in TMEM (2 x 256 fp32 columns) so the epilogue of
+// one tile overlaps the mainloop of the next.  The CTA is persistent over a tile list
+// derived on the device from the routing (per-expert token counts).
+// Every mbarrier wait is bounded (2 s); a timeout raises MOEQ_ERR_TIMEOUT and the CTA
+// drains its in-flight copies and MMAs, frees TMEM and returns.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moeq {
+
+constexpr int BM = 128;
+constexpr int BN = kTileN;  // 256
+constexpr int BK = 64;
+constexpr int kStages = 4;
+constexpr int kThreads = 320;
+constexpr int kGroupM = 16;  // m-tiles walked per token tile before moving on (L2 reuse)
+constexpr uint32_t kABytes = BM * BK * 2;
+constexpr uint32_t kBBytes = BN * BK * 2;
+constexpr uint32_t kLutBytes = 16 * 256;
+
+template <int MODE>
+struct Cfg {
+  static constexpr uint32_t kCodeRow = (MODE == MOEQ_INT8_ROW) ? 64 : 32;  // bytes/row/stage
+  static constexpr uint32_t kCodeBytes = BM * kCodeRow;
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes + kCodeBytes;
+  static constexpr uint32_t kLut = (MODE == MOEQ_INT8_ROW) ? 0 : kLutBytes;
+  static constexpr uint32_t kSmem = kStages * kStageBytes + kLut + 256 + 1024;
+};
+
+struct TmapSet {
+  CUtensorMap b[5];  // activation rows, boxes of 16, 32, 64, 128, 256 rows x 64 elements
+  CUtensorMap codes; // packed codes, [E*R rows, bytes per row], box 64 rows x kCodeRow
+};
+
+struct GemmArgs {
+  const float *absmax;      // NF4: [E*R, C/64]; INT8: [E*R]
+  const int8_t *aq;         // NF4_DQ
+  const float *ascale;      // NF4_DQ
+  const float *aoff;        // NF4_DQ
+  int E, R, C, I, MT, nk, nb, nblk;
+  const int32_t *offsets;
+  const int32_t *ntp;
+  const int32_t *perm;
+  __nv_bfloat16 *h_out;
+  float *slot_out;
+  const void *topk_w;
+  int w_bf16;
+  int32_t *status;
+};
+
+struct Tile {
+  int e, m, row0, count, nbox;
+};
+
+__device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a) {
+  int lo = 0, hi = a.E;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (a.ntp[mid] * a.MT <= tile) lo = mid;
+    else hi = mid;
+  }
+  Tile t;
+  t.e = lo;
+  const int NT = a.ntp[lo + 1] - a.ntp[lo];
+  const int local = tile - a.ntp[lo] * a.MT;
+  const int gfull = NT * kGroupM;
+  const int g = local / gfull;
+  const int rem = local - g * gfull;
+  const int Gg = min(kGroupM, a.MT - g * kGroupM);
+  const int nt = rem / Gg;
+  t.m = g * kGroupM + (rem - nt * Gg);
+  const int off = a.offsets[lo];
+  const int n_e = a.offsets[lo + 1] - off;
+  const int n0 = nt * BN;
+  t.count = min(BN, n_e - n0);
+  t.row0 = off + n0;
+  t.nbox = t.count <= 16 ? 0 : t.count <= 32 ? 1 : t.count <= 64 ? 2 : t.count <= 128 ? 3 : 4;
+  return t;
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts_u4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// fp32 absmax of weight row `wr` (expert e), NF4 block kb
+template <int MODE>
+__device__ __forceinline__ float load_absmax(const GemmArgs &a, int e, int wr, int kb) {
+  if (MODE == MOEQ_NF4) {
+    return __ldg(a.absmax + (static_cast<size_t>(e) * a.R + wr) * (a.C / 64) + kb);
+  } else if (MODE == MOEQ_NF4_DQ) {
+    const int b = wr * (a.C / 64) + kb;  // block index inside expert e
+    const float q = static_cast<float>(__ldg(a.aq + static_cast<size_t>(e) * a.nb + b));
+    const float s = __ldg(a.ascale + static_cast<size_t>(e) * a.nblk + (b >> 8));
+    return __fadd_rn(__fmul_rn(q, __fdiv_rn(s, 127.0f)), __ldg(a.aoff + e));
+  }
+  return 0.0f;
+}
+
+template <int MODE, int KIND>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_moe_gemm(const __grid_constant__ TmapSet maps, const GemmArgs args) {
+  using CF = Cfg<MODE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t lut = sbase + kStages * CF::kStageBytes;
+  uint8_t *ctrl = smem + kStages * CF::kStageBytes + CF::kLut;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl);
+  // bars: [0,4) tma_full, [4,8) a_full, [8,12) empty, [12,14) acc_full, [14,16) acc_empty, 16 drain
+  const uint32_t bar0 = smem_u32(bars);
+  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * i; };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ctrl + 17 * 8);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 17 * 8 + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(BAR(s), 1);           // tma_full: producer arrive + tx bytes
+      mbar_init(BAR(4 + s), 4);       // a_full: one arrival per dequant warp
+      mbar_init(BAR(8 + s), 1);       // empty: MMA commit
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(BAR(12 + b), 1);      // acc_full: MMA commit
+      mbar_init(BAR(14 + b), 4);      // acc_empty: one arrival per epilogue warp
+    }
+    mbar_init(BAR(16), 1);            // drain
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (MODE != MOEQ_INT8_ROW) {
+    // NF4 level table, one copy per lane: entry (code, lane) at code*256 + lane*4, so
+    // that each lane reads its own bank whatever code it looks up.
+    for (int i = threadIdx.x; i < 16 * 32; i += kThreads) {
+      const int code = i >> 5, l = i & 31;
+      const float cv[16] = {-1.0f, -0.6961928009986877f, -0.5250730514526367f, -0.39491748809814453f,
+                            -0.28444138169288635f, -0.18477343022823334f, -0.09105003625154495f, 0.0f,
+                            0.07958029955625534f, 0.16093020141124725f, 0.24611230194568634f,
+                            0.33791524171829224f, 0.44070982933044434f, 0.5626170039176941f,
+                            0.7229568362236023f, 1.0f};
+      *reinterpret_cast<float *>(smem + kStages * CF::kStageBytes + code * 256 + l * 4) = cv[code];
+    }
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    for (int i = 0; i < 5; ++i) tma_prefetch_desc(&maps.b[i]);
+    tma_prefetch_desc(&maps.codes);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int total_tiles = args.ntp[args.E] * args.MT;
+  const int nk = args.nk;
+
+  if (warp == 8) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        const Tile t = decode_tile(tile, args);
+        int y0, y1;
+        if (KIND == 0) {
+          y0 = t.e * args.R + t.m * 64;
+          y1 = y0 + args.I;
+        } else {
+          y0 = t.e * args.R + t.m * 128;
+          y1 = y0 + 64;
+        }
+        const uint32_t tx = (16u << t.nbox) * 128u + CF::kCodeBytes;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
+          if (!mbar_wait(BAR(8 + s), ph ^ 1u, abort_flag, args.status)) { ok = false; break; }
+          const uint32_t st = sbase + s * CF::kStageBytes;
+          mbar_arrive_expect_tx(BAR(s), tx);
+          tma_load_2d(st + kABytes, &maps.b[t.nbox], kb * BK, t.row0, BAR(s));
+          tma_load_2d(st + kABytes + kBBytes, &maps.codes, kb * CF::kCodeRow, y0, BAR(s));
+          tma_load_2d(st + kABytes + kBBytes + 64 * CF::kCodeRow, &maps.codes, kb * CF::kCodeRow, y1, BAR(s));
+        }
+      }
+      // drain: every copy issued lands before the CTA may exit
+      const uint32_t n = it < kStages ? it : kStages;
+      for (uint32_t d = 0; d < n; ++d) {
+        const uint32_t j = it - 1 - d;
+        uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(BAR(j % kStages), (j / kStages) & 1u)) {
+          if (globaltimer() - t0 > kWaitLimitNs) break;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      uint32_t it = 0, acc_it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++acc_it) {
+        const Tile t = decode_tile(tile, args);
+        const uint32_t b = acc_it & 1u, aph = (acc_it >> 1) & 1u;
+        if (!mbar_wait(BAR(14 + b), aph ^ 1u, abort_flag, args.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + b * 256u;
+        const uint32_t n_mma = static_cast<uint32_t>((t.count + 15) & ~15);
+        const uint32_t idesc = umma_idesc_bf16_m128(n_mma);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
+          if (!mbar_wait(BAR(s), ph, abort_flag, args.status) ||
+              !mbar_wait(BAR(4 + s), ph, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = sbase + s * CF::kStageBytes;
+          const uint64_t adesc = umma_desc_sw128(st);
+          const uint64_t bdesc = umma_desc_sw128(st + kABytes);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            // +32 bytes along K inside the 128-byte swizzle row = +2 in the start field
+            umma_bf16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          umma_commit(BAR(8 + s));
+        }
+        if (!ok) break;
+        umma_commit(BAR(12 + b));
+      }
+      // drain: all issued MMAs complete before TMEM is freed
+      umma_commit(BAR(16));
+      uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(BAR(16), 0)) {
+        if (globaltimer() - t0 > kWaitLimitNs) break;
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---------------- dequant ----------------
+    const int r = threadIdx.x - 128;  // tile row = TMEM lane = A row
+    const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      const Tile t = decode_tile(tile, args);
+      int wr, cr;  // weight row inside the expert, row inside the staged code tile
+      if (KIND == 0) {
+        const int sgate = r & 1, i = r >> 1;
+        wr = sgate * args.I + t.m * 64 + i;
+        cr = sgate * 64 + i;
+      } else {
+        wr = t.m * 128 + r;
+        cr = r;
+      }
+      float a_cur = 0.f, a_nxt = 0.f;
+      if (MODE != MOEQ_INT8_ROW) {
+        a_cur = load_absmax<MODE>(args, t.e, wr, 0);
+        if (nk > 1) a_nxt = load_absmax<MODE>(args, t.e, wr, 1);
+      }
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
+        float a_nn = 0.f;
+        if (MODE != MOEQ_INT8_ROW && kb + 2 < nk) a_nn = load_absmax<MODE>(args, t.e, wr, kb + 2);
+        if (!mbar_wait(BAR(s), ph, abort_flag, args.status)) { ok = false; break; }
+        const uint32_t st = sbase + s * CF::kStageBytes;
+        const uint32_t crow = st + kABytes + kBBytes + cr * CF::kCodeRow;
+        const uint32_t arow = st + r * 128;
+        const uint32_t sw = static_cast<uint32_t>(r & 7);
+        if (MODE == MOEQ_INT8_ROW) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const uint4 cw = lds_u4(crow + q4 * 16);
+            const uint32_t wv[4] = {cw.x, cw.y, cw.z, cw.w};
+            uint32_t o[8];
+#pragma unroll
+            for (int wi = 0; wi < 4; ++wi) {
+              const uint32_t bw = wv[wi] ^ 0x80808080u;  // byte = q + 128
+              float f[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                f[k] = __fsub_rn(__uint_as_float(__byte_perm(bw, 0x4B000000u, 0x7540u | k)), 8388736.0f);
+              o[2 * wi] = pack_bf16(f[0], f[1]);
+              o[2 * wi + 1] = pack_bf16(f[2], f[3]);
+            }
+            // 16 elements = two 16-byte chunks (2*q4, 2*q4+1)
+            sts_u4(arow + ((((2 * q4) ^ sw)) << 4), o[0], o[1], o[2], o[3]);
+            sts_u4(arow + ((((2 * q4 + 1) ^ sw)) << 4), o[4], o[5], o[6], o[7]);
+          }
+        } else {
+          const float a = a_cur;
+          const uint4 c0 = lds_u4(crow), c1 = lds_u4(crow + 16);
+          const uint32_t wv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t hi = (wv[j] >> 4) & 0x0F0F0F0Fu;  // even elements
+            const uint32_t lo = wv[j] & 0x0F0F0F0Fu;         // odd elements
+            uint32_t o[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t sel = 0x5504u | (static_cast<uint32_t>(k) << 4);
+              const float ce = __uint_as_float(lds_u32(lut + __byte_perm(hi, lane4, sel)));
+              const float co = __uint_as_float(lds_u32(lut + __byte_perm(lo, lane4, sel)));
+              o[k] = pack_bf16(__fmul_rn(ce, a), __fmul_rn(co, a));
+            }
+            sts_u4(arow + ((static_cast<uint32_t>(j) ^ sw) << 4), o[0], o[1], o[2], o[3]);
+          }
+          a_cur = a_nxt;
+          a_nxt = a_nn;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(4 + s));
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 0-3) ----------------
+    const int r = warp * 32 + lane;
+    uint32_t acc_it = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++acc_it) {
+      const Tile t = decode_tile(tile, args);
+      const uint32_t b = acc_it & 1u, aph = (acc_it >> 1) & 1u;
+      if (!mbar_wait(BAR(12 + b), aph, abort_flag, args.status)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + b * 256u;
+      const int nch = (t.count + 31) >> 5;
+      if (KIND == 0) {
+        const int sgate = lane & 1;
+        const int j = t.m * 64 + (r >> 1);
+        float step = 1.0f;
+        if (MODE == MOEQ_INT8_ROW)
+          step = __fdiv_rn(__ldg(args.absmax + static_cast<size_t>(t.e) * args.R + sgate * args.I + j), 127.0f);
+        for (int c = 0; c < nch; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tbase + c * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const float own = __uint_as_float(sgate ? v[16 + q] : v[q]) * step;
+            const float snd = __uint_as_float(sgate ? v[q] : v[16 + q]) * step;
+            const float rcv = __shfl_xor_sync(0xffffffffu, snd, 1);
+            const float g = sgate ? rcv : own;
+            const float u = sgate ? own : rcv;
+            const int col = c * 32 + (sgate ? 16 : 0) + q;
+            const float hval = g / (1.0f + __expf(-g)) * u;
+            if (col < t.count)
+              args.h_out[static_cast<size_t>(t.row0 + col) * args.I + j] = __float2bfloat16_rn(hval);
+          }
+        }
+      } else {
+        const int i = t.m * 128 + r;
+        float step = 1.0f;
+        if (MODE == MOEQ_INT8_ROW)
+          step = __fdiv_rn(__ldg(args.absmax + static_cast<size_t>(t.e) * args.R + i), 127.0f);
+        for (int c = 0; c < nch; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tbase + c * 32, v);
+          tmem_ld_wait();
+          const int colL = c * 32 + lane;
+          int p = 0;
+          float wv = 0.0f;
+          if (colL < t.count) {
+            p = __ldg(args.perm + t.row0 + colL);
+            if (args.w_bf16)
+              wv = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(args.topk_w)[p]);
+            else
+              wv = __ldg(reinterpret_cast<const float *>(args.topk_w) + p);
+          }
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const int pq = __shfl_sync(0xffffffffu, p, q);
+            const float wq = __shfl_sync(0xffffffffu, wv, q);
+            if (c * 32 + q < t.count)
+              args.slot_out[static_cast<size_t>(pq) * args.R + i] = wq * (__uint_as_float(v[q]) * step);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(14 + b));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+static bool encode_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner,
+                      uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                      CUtensorMapSwizzle sw) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE, int KIND>
+static cudaError_t launch_t(const TmapSet &maps, const GemmArgs &a, int grid, cudaStream_t s) {
+  using CF = Cfg<MODE>;
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(k_moe_gemm<MODE, KIND>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, CF::kSmem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  k_moe_gemm<MODE, KIND><<<grid, kThreads, CF::kSmem, s>>>(maps, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_moe_gemm(const GemmLaunch &g, int sm_count, cudaStream_t s, int *launches) {
+  const moeq_packed *w = g.w;
+  TmapSet maps;
+  const int C = w->C;
+  const uint32_t code_row = (g.mode == MOEQ_INT8_ROW) ? 64u : 32u;
+  for (int i = 0; i < 5; ++i) {
+    if (!encode_2d(&maps.b[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.act, C, g.S, static_cast<uint64_t>(C) * 2,
+                   64, 16u << i, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  const uint64_t row_bytes = (g.mode == MOEQ_INT8_ROW) ? C : C / 2;
+  if (!encode_2d(&maps.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, row_bytes,
+                 static_cast<uint64_t>(w->E) * w->R, row_bytes, code_row, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+
+  GemmArgs a;
+  a.absmax = w->absmax;
+  a.aq = w->absmax_q;
+  a.ascale = w->absmax_scale;
+  a.aoff = w->absmax_offset;
+  a.E = w->E;
+  a.R = w->R;
+  a.C = C;
+  a.I = g.I;
+  a.MT = (g.kind == 0) ? g.I / 64 : w->R / 128;
+  a.nk = C / 64;
+  a.nb = static_cast<int>(static_cast<long long>(w->R) * C / 64);
+  a.nblk = (a.nb + 255) / 256;
+  a.offsets = g.offsets;
+  a.ntp = g.ntile_prefix;
+  a.perm = g.perm;
+  a.h_out = static_cast<__nv_bfloat16 *>(g.h_out);
+  a.slot_out = g.slot_out;
+  a.topk_w = g.topk_w;
+  a.w_bf16 = g.w_bf16;
+  a.status = g.status;
+
+  const long long max_tiles = (static_cast<long long>(w->E) + (g.S + BN - 1) / BN) * a.MT;
+  const int grid = static_cast<int>(max_tiles < sm_count ? max_tiles : sm_count);
+  cudaError_t e;
+  if (g.mode == MOEQ_NF4) e = g.kind == 0 ? launch_t<MOEQ_NF4, 0>(maps, a, grid, s) : launch_t<MOEQ_NF4, 1>(maps, a, grid, s);
+  else if (g.mode == MOEQ_NF4_DQ) e = g.kind == 0 ? launch_t<MOEQ_NF4_DQ, 0>(maps, a, grid, s) : launch_t<MOEQ_NF4_DQ, 1>(maps, a, grid, s);
+  else e = g.kind == 0 ? launch_t<MOEQ_INT8_ROW, 0>(maps, a, grid, s) : launch_t<MOEQ_INT8_ROW, 1>(maps, a, grid, s);
+  ++*launches;
+  return e;
+}
+
+}  // namespace moeq

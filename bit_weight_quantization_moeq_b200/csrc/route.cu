@@ -1,0 +1,226 @@
+// Routing of the (t, k) pairs to experts, activation gather and the k-ordered combine.
+//
+// The experts interface is (hidden_states, top_k_index, top_k_weights) (unsloth-zoo
+// issue #850).  Grouping: counts[e] = #pairs routed to e, offsets = exclusive prefix
+// sum, perm = the flat pair index p = t*K + k listed by expert and in increasing p
+// within an expert (stable).  A pair whose index is outside [0, E) is dropped.
+//
+// Work is cut into chunks of kRouteChunk consecutive pairs, one warp per chunk, so
+// that the stable order comes from walking each chunk in order (32 pairs at a time,
+// ranks inside a step from __match_any_sync) and from chunk bases taken in chunk order.
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moeq {
+
+constexpr int kWarpsPerBlock = 8;
+constexpr int kSteps = kRouteChunk / 32;
+
+template <typename IdxT>
+__device__ __forceinline__ int load_expert(const IdxT *idx, int p, int S, int E, int32_t *status) {
+  if (p >= S) return -1;
+  const long long e = static_cast<long long>(idx[p]);
+  if (e < 0 || e >= E) {
+    report(status, MOEQ_ERR_INDEX);
+    return -1;
+  }
+  return static_cast<int>(e);
+}
+
+// Per-chunk histograms counts_chunk[chunk][e].
+template <typename IdxT>
+__global__ void __launch_bounds__(256) k_route_count(const IdxT *__restrict__ idx, int S, int E,
+                                                     int nchunks, int32_t *__restrict__ counts_chunk,
+                                                     int32_t *status) {
+  extern __shared__ int32_t hist[];  // [kWarpsPerBlock][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x * kWarpsPerBlock + warp;
+  if (chunk >= nchunks) return;  // whole warp; no block-wide barrier below
+  int32_t *h = hist + warp * E;
+  for (int e = lane; e < E; e += 32) h[e] = 0;
+  __syncwarp();
+  for (int st = 0; st < kSteps; ++st) {
+    const int p = chunk * kRouteChunk + st * 32 + lane;
+    const int e = load_expert(idx, p, S, E, status);
+    if (e >= 0) atomicAdd(&h[e], 1);
+  }
+  __syncwarp();
+  int32_t *dst = counts_chunk + static_cast<size_t>(chunk) * E;
+  for (int e = lane; e < E; e += 32) dst[e] = h[e];
+}
+
+// Exclusive scan of one value per thread over the block (blockDim.x == 1024).
+__device__ int block_exclusive_scan(int v, int *warp_tot, int *total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, d);
+    if (lane >= d) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_tot[lane];
+    int z = w;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, z, d);
+      if (lane >= d) z += y;
+    }
+    warp_tot[lane] = z - w;  // exclusive prefix of warp totals
+    if (lane == 31) *total = z;
+  }
+  __syncthreads();
+  const int r = warp_tot[warp] + x - v;
+  __syncthreads();
+  return r;
+}
+
+// Totals per expert, offsets, tile prefix and per-(chunk, expert) bases.
+__global__ void __launch_bounds__(1024) k_route_scan(const int32_t *__restrict__ counts_chunk,
+                                                     int nchunks, int E,
+                                                     int32_t *__restrict__ chunk_base,
+                                                     int32_t *__restrict__ counts,
+                                                     int32_t *__restrict__ offsets,
+                                                     int32_t *__restrict__ ntile_prefix) {
+  __shared__ int warp_tot[32];
+  __shared__ int total_cnt, total_tiles;
+  const int e = threadIdx.x;
+  int tot = 0;
+  if (e < E) {
+    for (int c = 0; c < nchunks; ++c) {
+      const size_t at = static_cast<size_t>(c) * E + e;
+      const int v = counts_chunk[at];
+      chunk_base[at] = tot;
+      tot += v;
+    }
+  }
+  const int off = block_exclusive_scan(tot, warp_tot, &total_cnt);
+  const int nt = (tot + kTileN - 1) / kTileN;
+  const int ntp = block_exclusive_scan(nt, warp_tot, &total_tiles);
+  if (e < E) {
+    offsets[e] = off;
+    ntile_prefix[e] = ntp;
+    if (counts) counts[e] = tot;
+    for (int c = 0; c < nchunks; ++c) chunk_base[static_cast<size_t>(c) * E + e] += off;
+  }
+  if (e == 0) {
+    offsets[E] = total_cnt;
+    ntile_prefix[E] = total_tiles;
+  }
+}
+
+// Stable scatter of pair indices into perm.
+template <typename IdxT>
+__global__ void __launch_bounds__(256) k_route_scatter(const IdxT *__restrict__ idx, int S, int E,
+                                                       int nchunks,
+                                                       const int32_t *__restrict__ chunk_base,
+                                                       int32_t *__restrict__ perm) {
+  extern __shared__ int32_t running_all[];  // [kWarpsPerBlock][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x * kWarpsPerBlock + warp;
+  if (chunk >= nchunks) return;
+  int32_t *running = running_all + warp * E;
+  const int32_t *base = chunk_base + static_cast<size_t>(chunk) * E;
+  for (int e = lane; e < E; e += 32) running[e] = base[e];
+  __syncwarp();
+  const unsigned lt = (1u << lane) - 1u;
+  for (int st = 0; st < kSteps; ++st) {
+    const int p = chunk * kRouteChunk + st * 32 + lane;
+    const int e = load_expert(idx, p, S, E, nullptr);
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0) {
+      const int rank = __popc(peers & lt);
+      perm[running[e] + rank] = p;
+    }
+    __syncwarp();
+    if (e >= 0 && (peers & lt) == 0) running[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+cudaError_t launch_route(const void *idx, bool idx64, int S, int E, int nchunks,
+                         int32_t *counts_chunk, int32_t *chunk_base, int32_t *counts,
+                         int32_t *offsets, int32_t *ntile_prefix, int32_t *perm, int32_t *status,
+                         cudaStream_t s, int *launches) {
+  const int blocks = (nchunks + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  const size_t shm = static_cast<size_t>(kWarpsPerBlock) * E * sizeof(int32_t);
+  if (idx64) k_route_count<long long><<<blocks, 256, shm, s>>>(static_cast<const long long *>(idx), S, E, nchunks, counts_chunk, status);
+  else k_route_count<int32_t><<<blocks, 256, shm, s>>>(static_cast<const int32_t *>(idx), S, E, nchunks, counts_chunk, status);
+  k_route_scan<<<1, 1024, 0, s>>>(counts_chunk, nchunks, E, chunk_base, counts, offsets, ntile_prefix);
+  if (idx64) k_route_scatter<long long><<<blocks, 256, shm, s>>>(static_cast<const long long *>(idx), S, E, nchunks, chunk_base, perm);
+  else k_route_scatter<int32_t><<<blocks, 256, shm, s>>>(static_cast<const int32_t *>(idx), S, E, nchunks, chunk_base, perm);
+  *launches += 3;
+  return cudaGetLastError();
+}
+
+// xg[s] = x[perm[s] / K] for s < offsets[E]: one warp per row, 16-byte vectors.
+__global__ void __launch_bounds__(256) k_gather_rows(const uint4 *__restrict__ x,
+                                                     const int32_t *__restrict__ perm,
+                                                     const int32_t *__restrict__ offsets, int E,
+                                                     int S, int K, int vec_per_row,
+                                                     uint4 *__restrict__ xg) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= S || row >= offsets[E]) return;
+  const int t = perm[row] / K;
+  const uint4 *src = x + static_cast<size_t>(t) * vec_per_row;
+  uint4 *dst = xg + static_cast<size_t>(row) * vec_per_row;
+  for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
+}
+
+cudaError_t launch_gather_rows(const void *x, const int32_t *perm, const int32_t *offsets, int E,
+                               int S, int K, int H, void *xg, cudaStream_t s, int *launches) {
+  const int blocks = (S + 7) / 8;
+  k_gather_rows<<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(x), perm, offsets, E, S, K, H / 8,
+                                       static_cast<uint4 *>(xg));
+  ++*launches;
+  return cudaGetLastError();
+}
+
+// out[t, i] = bf16( sum over k = 0..K-1 in order of slots[t*K + k, i] ), skipping
+// dropped pairs.  One thread per 8 features.
+template <typename IdxT>
+__global__ void __launch_bounds__(256) k_combine(const float4 *__restrict__ slots,
+                                                 const IdxT *__restrict__ idx, int T, int K, int E,
+                                                 int H8, uint4 *__restrict__ out) {
+  const size_t g = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (g >= static_cast<size_t>(T) * H8) return;
+  const size_t t = g / H8, j = g - t * H8;
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int k = 0; k < K; ++k) {
+    const long long e = static_cast<long long>(idx[t * K + k]);
+    if (e < 0 || e >= E) continue;
+    const float4 *src = slots + ((t * K + k) * H8 + j) * 2;
+    const float4 a = src[0], b = src[1];
+    acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+    acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+  }
+  uint32_t p[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+    p[i] = *reinterpret_cast<const uint32_t *>(&h);
+  }
+  out[g] = make_uint4(p[0], p[1], p[2], p[3]);
+}
+
+cudaError_t launch_combine(const float *slots, const void *idx, bool idx64, int T, int K, int E,
+                           int H, void *out, cudaStream_t s, int *launches) {
+  const int H8 = H / 8;
+  const size_t n = static_cast<size_t>(T) * H8;
+  const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
+  const float4 *sp = reinterpret_cast<const float4 *>(slots);
+  uint4 *op = static_cast<uint4 *>(out);
+  if (idx64) k_combine<long long><<<blocks, 256, 0, s>>>(sp, static_cast<const long long *>(idx), T, K, E, H8, op);
+  else k_combine<int32_t><<<blocks, 256, 0, s>>>(sp, static_cast<const int32_t *>(idx), T, K, E, H8, op);
+  ++*launches;
+  return cudaGetLastError();
+}
+
+}  // namespace moeq
