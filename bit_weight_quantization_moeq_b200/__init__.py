@@ -26,7 +26,8 @@ MOEQ_NF4, MOEQ_NF4_DQ, MOEQ_INT8_ROW = 0, 1, 2
 MOEQ_BF16, MOEQ_F32, MOEQ_I32, MOEQ_I64 = 0, 1, 2, 3
 STATUS = {0: "MOEQ_OK", 1: "MOEQ_ERR_NULL", 2: "MOEQ_ERR_SHAPE", 3: "MOEQ_ERR_DTYPE",
           4: "MOEQ_ERR_ALIGN", 5: "MOEQ_ERR_BLOCKSIZE", 6: "MOEQ_ERR_WORKSPACE",
-          7: "MOEQ_ERR_CUDA", 8: "MOEQ_ERR_TIMEOUT", 9: "MOEQ_ERR_INDEX", 10: "MOEQ_ERR_DEVICE"}
+          7: "MOEQ_ERR_CUDA", 8: "MOEQ_ERR_TIMEOUT", 9: "MOEQ_ERR_INDEX", 10: "MOEQ_ERR_DEVICE",
+          11: "MOEQ_ERR_RANGE"}
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoeq.so")
 if not os.path.exists(LIB_PATH):
@@ -53,7 +54,7 @@ _sigs = {
     "moeq_quantize_nf4": (_i, [_vp, _i, _i, _i, _i, _P, _vp, _sz, _vp]),
     "moeq_quantize_int8_rowwise": (_i, [_vp, _i, _i, _i, _P, _vp]),
     "moeq_dequantize": (_i, [_P, _vp, _i, _vp]),
-    "moeq_experts_forward": (_i, [_vp, _vp, _i, _vp, _i, _i, _i, _P, _P, _vp, _vp, _sz, _vp, _vp]),
+    "moeq_experts_forward": (_i, [_vp, _vp, _i, _vp, _i, _i, _i, _P, _P, _vp, _i, _vp, _sz, _vp, _vp]),
     "moeq_route": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
     "moeq_status_string": (ctypes.c_char_p, [_i]),
     "moeq_set_trace_events": (None, [ctypes.POINTER(ctypes.c_void_p), _i]),
@@ -232,19 +233,20 @@ def moeq_route(top_k_index: torch.Tensor, E: int, ws: torch.Tensor | None = None
 def moeq_experts_forward(hidden: torch.Tensor, top_k_index: torch.Tensor, top_k_weights: torch.Tensor,
                          gate_up: PackedWeight, down: PackedWeight, out: torch.Tensor | None = None,
                          ws: torch.Tensor | None = None, d_status: torch.Tensor | None = None,
-                         stream=None) -> torch.Tensor:
+                         stream=None, out_dtype=torch.bfloat16) -> torch.Tensor:
     T, H = hidden.shape
     K = top_k_index.shape[1]
     I = down.C
     dev = hidden.device
     if out is None:
-        out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        out = torch.empty((T, H), dtype=out_dtype, device=dev)
     if ws is None:
         ws = torch.empty(max(moeq_forward_workspace(T, K, gate_up.E, H, I), 16), dtype=torch.uint8, device=dev)
+    odt = MOEQ_F32 if out.dtype == torch.float32 else MOEQ_BF16
     idt = MOEQ_I64 if top_k_index.dtype == torch.int64 else MOEQ_I32
     wdt = MOEQ_BF16 if top_k_weights.dtype == torch.bfloat16 else MOEQ_F32
     dg, dd = gate_up.descriptor(), down.descriptor()
     _check(lib.moeq_experts_forward(_ptr(hidden), _ptr(top_k_index), idt, _ptr(top_k_weights), wdt, T, K,
-                                    ctypes.byref(dg), ctypes.byref(dd), _ptr(out), _ptr(ws), ws.numel(),
+                                    ctypes.byref(dg), ctypes.byref(dd), _ptr(out), odt, _ptr(ws), ws.numel(),
                                     _ptr(d_status), _stream(stream)), "moeq_experts_forward")
     return out

@@ -274,9 +274,11 @@ moeq_status moeq_route(const void *top_k_index, int index_dtype, int T, int K, i
 
 moeq_status moeq_experts_forward(const void *hidden, const void *top_k_index, int index_dtype,
                                  const void *top_k_weights, int weight_dtype, int T, int K,
-                                 const moeq_packed *gate_up, const moeq_packed *down, void *out, void *ws,
-                                 size_t ws_bytes, int32_t *d_status, moeq_stream_t stream) {
+                                 const moeq_packed *gate_up, const moeq_packed *down, void *out,
+                                 int out_dtype, void *ws, size_t ws_bytes, int32_t *d_status,
+                                 moeq_stream_t stream) {
   if (T < 0 || K <= 0) return MOEQ_ERR_SHAPE;
+  if (out_dtype != MOEQ_BF16 && out_dtype != MOEQ_F32) return MOEQ_ERR_DTYPE;
   if (index_dtype != MOEQ_I32 && index_dtype != MOEQ_I64) return MOEQ_ERR_DTYPE;
   if (weight_dtype != MOEQ_F32 && weight_dtype != MOEQ_BF16) return MOEQ_ERR_DTYPE;
   moeq_status st;
@@ -312,7 +314,7 @@ moeq_status moeq_experts_forward(const void *hidden, const void *top_k_index, in
   void *xg = at<void>(ws, l.xg);
   void *h = at<void>(ws, l.h);
   float *slots = at<float>(ws, l.slots);
-  if (e == cudaSuccess) e = launch_gather_rows(hidden, perm, offsets, E, S, K, H, xg, s, &launches);
+  if (e == cudaSuccess) e = launch_gather_rows(hidden, perm, offsets, E, S, K, H, xg, status, s, &launches);
   trace_mark(2, s);
   if (e == cudaSuccess) {
     GemmLaunch g{};
@@ -348,7 +350,8 @@ moeq_status moeq_experts_forward(const void *hidden, const void *top_k_index, in
     e = launch_moe_gemm(g, di.sm_count, s, &launches);
   }
   trace_mark(4, s);
-  if (e == cudaSuccess) e = launch_combine(slots, top_k_index, index_dtype == MOEQ_I64, T, K, E, H, out, s, &launches);
+  if (e == cudaSuccess) e = launch_combine(slots, top_k_index, index_dtype == MOEQ_I64, T, K, E, H, out, out_dtype == MOEQ_F32, s,
+                                          &launches);
   trace_mark(5, s);
   return finish(e, launches);
 }
@@ -366,6 +369,7 @@ const char *moeq_status_string(moeq_status s) {
     case MOEQ_ERR_TIMEOUT: return "device pipeline wait timed out";
     case MOEQ_ERR_INDEX: return "top_k_index out of range (pair dropped)";
     case MOEQ_ERR_DEVICE: return "device is not sm_100 (B200)";
+    case MOEQ_ERR_RANGE: return "activation beyond fp16 range was saturated";
   }
   return "unknown status";
 }

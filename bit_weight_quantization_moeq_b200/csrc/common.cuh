@@ -115,8 +115,8 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (bf16 in, fp32 accumulate)
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (16-bit in, fp32 accumulate)
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                           uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -150,7 +150,7 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 // Shared-memory matrix descriptor for a K-major operand tile stored with the
-// 128-byte swizzle: rows of 64 bf16 (128 B), 8-row groups 1024 B apart, tile base
+// 128-byte swizzle: rows of 64 16-bit elements (128 B), 8-row groups 1024 B apart, tile base
 // 1024-byte aligned.  Bits: start>>4 [0,14), LBO>>4 [16,30) (unused for swizzled
 // K-major, set to 1), SBO>>4 [32,46) = 1024>>4, fixed version 1 at [46,48),
 // base offset 0, layout type 2 (128B swizzle) at [61,64).
@@ -164,12 +164,12 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr) {
   return d;
 }
 
-// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both K-major,
-// M = 128, N = n (multiple of 16, 16..256).
-__device__ __forceinline__ uint32_t umma_idesc_bf16_m128(uint32_t n) {
+// Instruction descriptor, kind::f16: fp32 accumulator, fp16 A and B (format code 0;
+// bf16 would be 1 for both), both K-major, M = 128, N = n (multiple of 16, 16..256).
+__device__ __forceinline__ uint32_t umma_idesc_f16_m128(uint32_t n) {
   return (1u << 4)               // D format: f32
-         | (1u << 7)             // A format: bf16
-         | (1u << 10)            // B format: bf16
+         | (0u << 7)             // A format: f16
+         | (0u << 10)            // B format: f16
          | ((n >> 3) << 17)      // N >> 3
          | ((128u >> 4) << 24);  // M >> 4
 }

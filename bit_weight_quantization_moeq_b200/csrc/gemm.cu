@@ -11,9 +11,10 @@
 // over the expert-sorted rows s of each expert e.
 //
 // Tile = 128 weight rows (UMMA M, operand A) x up to 256 tokens (UMMA N, operand B) x
-// K in steps of 64 (one NF4 block, one 128-byte swizzle row).
+// K in steps of 64 (one NF4 block, one 128-byte swizzle row).  Both operands are fp16
+// (weights dequantized to fp16, activations and h stored as fp16), accumulation fp32.
 //   warps 0-3  epilogue: TMEM -> registers (tcgen05.ld), SiLU*up or weighted slot stores
-//   warps 4-7  dequant: packed codes (TMA'd into SMEM) -> bf16 A tile in the UMMA
+//   warps 4-7  dequant: packed codes (TMA'd into SMEM) -> fp16 A tile in the UMMA
 //              K-major 128B-swizzled layout, one weight row per thread
 //   warp 8     producer: TMA of the token tile (B, 128B swizzle) and of the code tiles
 //   warp 9     TMEM allocation and the single-thread tcgen05.mma issue
@@ -26,6 +27,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -65,7 +67,7 @@ struct GemmArgs {
   const int32_t *offsets;
   const int32_t *ntp;
   const int32_t *perm;
-  __nv_bfloat16 *h_out;
+  __half *h_out;
   float *slot_out;
   const void *topk_w;
   int w_bf16;
@@ -118,8 +120,8 @@ __device__ __forceinline__ void sts_u4(uint32_t addr, uint32_t a, uint32_t b, ui
   asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
 }
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t *>(&h);
 }
 
@@ -247,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * 256u;
         const uint32_t n_mma = static_cast<uint32_t>((t.count + 15) & ~15);
-        const uint32_t idesc = umma_idesc_bf16_m128(n_mma);
+        const uint32_t idesc = umma_idesc_f16_m128(n_mma);
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
           if (!mbar_wait(BAR(s), ph, abort_flag, args.status) ||
@@ -262,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             // +32 bytes along K inside the 128-byte swizzle row = +2 in the start field
-            umma_bf16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
+            umma_f16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
           }
           umma_commit(BAR(8 + s));
         }
@@ -321,8 +323,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int k = 0; k < 4; ++k)
                 f[k] = __fsub_rn(__uint_as_float(__byte_perm(bw, 0x4B000000u, 0x7540u | k)), 8388736.0f);
-              o[2 * wi] = pack_bf16(f[0], f[1]);
-              o[2 * wi + 1] = pack_bf16(f[2], f[3]);
+              o[2 * wi] = pack_f16(f[0], f[1]);
+              o[2 * wi + 1] = pack_f16(f[2], f[3]);
             }
             // 16 elements = two 16-byte chunks (2*q4, 2*q4+1)
             sts_u4(arow + ((((2 * q4) ^ sw)) << 4), o[0], o[1], o[2], o[3]);
@@ -342,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t sel = 0x5504u | (static_cast<uint32_t>(k) << 4);
               const float ce = __uint_as_float(lds_u32(lut + __byte_perm(hi, lane4, sel)));
               const float co = __uint_as_float(lds_u32(lut + __byte_perm(lo, lane4, sel)));
-              o[k] = pack_bf16(__fmul_rn(ce, a), __fmul_rn(co, a));
+              o[k] = pack_f16(__fmul_rn(ce, a), __fmul_rn(co, a));
             }
             sts_u4(arow + ((static_cast<uint32_t>(j) ^ sw) << 4), o[0], o[1], o[2], o[3]);
           }
@@ -383,9 +385,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float g = sgate ? rcv : own;
             const float u = sgate ? own : rcv;
             const int col = c * 32 + (sgate ? 16 : 0) + q;
-            const float hval = g / (1.0f + __expf(-g)) * u;
-            if (col < t.count)
-              args.h_out[static_cast<size_t>(t.row0 + col) * args.I + j] = __float2bfloat16_rn(hval);
+            float hval = g / (1.0f + __expf(-g)) * u;
+            if (col < t.count) {
+              if (fabsf(hval) > 65504.0f) {
+                report(args.status, MOEQ_ERR_RANGE);
+                hval = fminf(fmaxf(hval, -65504.0f), 65504.0f);
+              }
+              args.h_out[static_cast<size_t>(t.row0 + col) * args.I + j] = __float2half_rn(hval);
+            }
           }
         }
       } else {
@@ -483,7 +490,7 @@ cudaError_t launch_moe_gemm(const GemmLaunch &g, int sm_count, cudaStream_t s, i
   const int C = w->C;
   const uint32_t code_row = (g.mode == MOEQ_INT8_ROW) ? 64u : 32u;
   for (int i = 0; i < 5; ++i) {
-    if (!encode_2d(&maps.b[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.act, C, g.S, static_cast<uint64_t>(C) * 2,
+    if (!encode_2d(&maps.b[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g.act, C, g.S, static_cast<uint64_t>(C) * 2,
                    64, 16u << i, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
@@ -508,7 +515,7 @@ cudaError_t launch_moe_gemm(const GemmLaunch &g, int sm_count, cudaStream_t s, i
   a.offsets = g.offsets;
   a.ntp = g.ntile_prefix;
   a.perm = g.perm;
-  a.h_out = static_cast<__nv_bfloat16 *>(g.h_out);
+  a.h_out = static_cast<__half *>(g.h_out);
   a.slot_out = g.slot_out;
   a.topk_w = g.topk_w;
   a.w_bf16 = g.w_bf16;

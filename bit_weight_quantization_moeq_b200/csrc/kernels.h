@@ -27,9 +27,10 @@ cudaError_t launch_route(const void *idx, bool idx64, int S, int E, int nchunks,
                          int32_t *offsets, int32_t *ntile_prefix, int32_t *perm, int32_t *status,
                          cudaStream_t s, int *launches);
 cudaError_t launch_gather_rows(const void *x, const int32_t *perm, const int32_t *offsets, int E,
-                               int S, int K, int H, void *xg, cudaStream_t s, int *launches);
+                               int S, int K, int H, void *xg, int32_t *status, cudaStream_t s,
+                               int *launches);
 cudaError_t launch_combine(const float *slots, const void *idx, bool idx64, int T, int K, int E,
-                           int H, void *out, cudaStream_t s, int *launches);
+                           int H, void *out, bool f32_out, cudaStream_t s, int *launches);
 
 // gemm.cu
 struct GemmLaunch {
@@ -38,9 +39,9 @@ struct GemmLaunch {
   const moeq_packed *w;
   int I;          // intermediate size (gate_up: R = 2I; down: C = I)
   int S;          // rows of the activation operand (T*K)
-  const void *act;  // bf16 [S, C] activation rows in expert-sorted order
+  const void *act;  // fp16 [S, C] activation rows in expert-sorted order
   const int32_t *offsets, *ntile_prefix, *perm;
-  void *h_out;      // gate_up: bf16 [S, I]
+  void *h_out;      // gate_up: fp16 [S, I]
   float *slot_out;  // down: f32 [T*K, H]
   const void *topk_w;
   int w_bf16;

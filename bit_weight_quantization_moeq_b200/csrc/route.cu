@@ -11,6 +11,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -159,36 +160,58 @@ cudaError_t launch_route(const void *idx, bool idx64, int S, int E, int nchunks,
   return cudaGetLastError();
 }
 
-// xg[s] = x[perm[s] / K] for s < offsets[E]: one warp per row, 16-byte vectors.
+// xg[s] = fp16(x[perm[s] / K]) for s < offsets[E]: one warp per row, 16-byte vectors.
+// bf16 -> fp16 is exact for 6.1e-5 <= |x| <= 65504; larger magnitudes saturate to
+// +-65504 and raise MOEQ_ERR_RANGE.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_sat(uint32_t w, bool &over) {
+  float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xffff0000u);
+  over |= (fabsf(lo) > 65504.0f) || (fabsf(hi) > 65504.0f);
+  lo = fminf(fmaxf(lo, -65504.0f), 65504.0f);
+  hi = fminf(fmaxf(hi, -65504.0f), 65504.0f);
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
+
 __global__ void __launch_bounds__(256) k_gather_rows(const uint4 *__restrict__ x,
                                                      const int32_t *__restrict__ perm,
                                                      const int32_t *__restrict__ offsets, int E,
                                                      int S, int K, int vec_per_row,
-                                                     uint4 *__restrict__ xg) {
+                                                     uint4 *__restrict__ xg, int32_t *status) {
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= S || row >= offsets[E]) return;
   const int t = perm[row] / K;
   const uint4 *src = x + static_cast<size_t>(t) * vec_per_row;
   uint4 *dst = xg + static_cast<size_t>(row) * vec_per_row;
-  for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
+  bool over = false;
+  for (int v = lane; v < vec_per_row; v += 32) {
+    const uint4 a = src[v];
+    uint4 b;
+    b.x = bf16x2_to_f16x2_sat(a.x, over);
+    b.y = bf16x2_to_f16x2_sat(a.y, over);
+    b.z = bf16x2_to_f16x2_sat(a.z, over);
+    b.w = bf16x2_to_f16x2_sat(a.w, over);
+    dst[v] = b;
+  }
+  if (over) report(status, MOEQ_ERR_RANGE);
 }
 
 cudaError_t launch_gather_rows(const void *x, const int32_t *perm, const int32_t *offsets, int E,
-                               int S, int K, int H, void *xg, cudaStream_t s, int *launches) {
+                               int S, int K, int H, void *xg, int32_t *status, cudaStream_t s,
+                               int *launches) {
   const int blocks = (S + 7) / 8;
   k_gather_rows<<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(x), perm, offsets, E, S, K, H / 8,
-                                       static_cast<uint4 *>(xg));
+                                       static_cast<uint4 *>(xg), status);
   ++*launches;
   return cudaGetLastError();
 }
 
-// out[t, i] = bf16( sum over k = 0..K-1 in order of slots[t*K + k, i] ), skipping
-// dropped pairs.  One thread per 8 features.
-template <typename IdxT>
+// out[t, i] = sum over k = 0..K-1, in order, of slots[t*K + k, i] (fp32), skipping
+// dropped pairs; stored as fp32 or rounded once to bf16.  One thread per 8 features.
+template <typename IdxT, bool F32OUT>
 __global__ void __launch_bounds__(256) k_combine(const float4 *__restrict__ slots,
                                                  const IdxT *__restrict__ idx, int T, int K, int E,
-                                                 int H8, uint4 *__restrict__ out) {
+                                                 int H8, void *__restrict__ out) {
   const size_t g = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (g >= static_cast<size_t>(T) * H8) return;
   const size_t t = g / H8, j = g - t * H8;
@@ -201,24 +224,33 @@ __global__ void __launch_bounds__(256) k_combine(const float4 *__restrict__ slot
     acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
     acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
   }
-  uint32_t p[4];
+  if (F32OUT) {
+    float4 *o = reinterpret_cast<float4 *>(out) + g * 2;
+    o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  } else {
+    uint32_t p[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-    p[i] = *reinterpret_cast<const uint32_t *>(&h);
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+      p[i] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    reinterpret_cast<uint4 *>(out)[g] = make_uint4(p[0], p[1], p[2], p[3]);
   }
-  out[g] = make_uint4(p[0], p[1], p[2], p[3]);
 }
 
 cudaError_t launch_combine(const float *slots, const void *idx, bool idx64, int T, int K, int E,
-                           int H, void *out, cudaStream_t s, int *launches) {
+                           int H, void *out, bool f32_out, cudaStream_t s, int *launches) {
   const int H8 = H / 8;
   const size_t n = static_cast<size_t>(T) * H8;
   const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
   const float4 *sp = reinterpret_cast<const float4 *>(slots);
-  uint4 *op = static_cast<uint4 *>(out);
-  if (idx64) k_combine<long long><<<blocks, 256, 0, s>>>(sp, static_cast<const long long *>(idx), T, K, E, H8, op);
-  else k_combine<int32_t><<<blocks, 256, 0, s>>>(sp, static_cast<const int32_t *>(idx), T, K, E, H8, op);
+  const long long *i64 = static_cast<const long long *>(idx);
+  const int32_t *i32 = static_cast<const int32_t *>(idx);
+  if (idx64 && f32_out) k_combine<long long, true><<<blocks, 256, 0, s>>>(sp, i64, T, K, E, H8, out);
+  else if (idx64) k_combine<long long, false><<<blocks, 256, 0, s>>>(sp, i64, T, K, E, H8, out);
+  else if (f32_out) k_combine<int32_t, true><<<blocks, 256, 0, s>>>(sp, i32, T, K, E, H8, out);
+  else k_combine<int32_t, false><<<blocks, 256, 0, s>>>(sp, i32, T, K, E, H8, out);
   ++*launches;
   return cudaGetLastError();
 }

@@ -32,7 +32,11 @@
  *   of gate_up, never inferred from the shape):
  *     out[t] = sum_k w[t,k] * down_e( silu(gate_e x_t) * up_e x_t ),  e = idx[t,k],
  *   with silu(z) = z / (1 + exp(-z)), fp32 accumulation, the k terms added in k
- *   order, the result rounded once to bf16.  top_k_weights are used as given.
+ *   order, the result rounded once to bf16.  top_k_weights are used as given.  The
+ *   tensor-core operands are fp16 (the compute dtype of the pages' bitsandbytes
+ *   reproduction, bnb_4bit_compute_dtype=float16): the dequantized weights, the
+ *   hidden rows (converted from bf16, exact for 6.1e-5 <= |x| <= 65504) and the
+ *   intermediate h; larger magnitudes saturate and report MOEQ_ERR_RANGE.
  *
  * Conventions (every entry point):
  *   - Memory: every pointer argument is a DEVICE pointer, 16-byte aligned, unless the
@@ -74,7 +78,9 @@ typedef enum {
   MOEQ_ERR_CUDA = 7,       /* a CUDA call or kernel launch failed */
   MOEQ_ERR_TIMEOUT = 8,    /* device: a pipeline wait ran past its limit (a bug) */
   MOEQ_ERR_INDEX = 9,      /* device: a top_k_index value outside [0, E) was dropped */
-  MOEQ_ERR_DEVICE = 10     /* the current device is not compute capability 10.0 */
+  MOEQ_ERR_DEVICE = 10,    /* the current device is not compute capability 10.0 */
+  MOEQ_ERR_RANGE = 11      /* device: an activation (hidden or h) beyond the fp16 range of
+                              the tensor-core operands (|v| > 65504) was saturated */
 } moeq_status;
 
 typedef enum { MOEQ_NF4 = 0, MOEQ_NF4_DQ = 1, MOEQ_INT8_ROW = 2 } moeq_mode;
@@ -137,7 +143,8 @@ size_t moeq_forward_workspace(int T, int K, int E, int H, int I);
  *   top_k_weights [T, K], fp32 (weight_dtype MOEQ_F32) or bf16 (MOEQ_BF16)
  *   gate_up       packed [E, 2I, H];  down: packed [E, H, I]; same mode and E
  *                 (modes NF4, NF4_DQ or INT8_ROW; H % 128 == 0, I % 64 == 0)
- *   out           bf16 [T, H] (fully overwritten)
+ *   out           [T, H], fully overwritten: bf16 (out_dtype MOEQ_BF16, the fp32 sum
+ *                 rounded once, to nearest even) or fp32 (MOEQ_F32, the sum itself)
  *   ws            device workspace of at least moeq_forward_workspace(T, K, E, H, I)
  *   d_status      optional device int32, zeroed by the caller: when the device finds
  *                 bad data it writes a moeq_status code there if the word is still 0
@@ -146,8 +153,8 @@ size_t moeq_forward_workspace(int T, int K, int E, int H, int I);
 moeq_status moeq_experts_forward(const void *hidden, const void *top_k_index, int index_dtype,
                                  const void *top_k_weights, int weight_dtype, int T, int K,
                                  const moeq_packed *gate_up, const moeq_packed *down,
-                                 void *out, void *ws, size_t ws_bytes, int32_t *d_status,
-                                 moeq_stream_t stream);
+                                 void *out, int out_dtype, void *ws, size_t ws_bytes,
+                                 int32_t *d_status, moeq_stream_t stream);
 
 /* Routing step of the forward on its own (the grouping of the (t, k) pairs by
  * expert): counts [E] (int32), offsets [E+1] (int32, exclusive prefix sum of counts)

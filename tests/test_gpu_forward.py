@@ -35,11 +35,17 @@ def make_inputs(E, H, I, T, K, seed, outliers=False, device="cuda"):
 
 
 def run_forward(inp, mode, **kw):
+    """fp32-output forward (the parity subject) and a check that the bf16 output of the
+    same call sequence is exactly the round-to-nearest-even of that fp32 output."""
     m = moeq()
     gu = quantize(inp["gate_up"], mode)
     dn = quantize(inp["down"], mode)
-    out = m.moeq_experts_forward(inp["hidden"], inp["top_k_index"], inp["top_k_weights"], gu, dn, **kw)
+    out = m.moeq_experts_forward(inp["hidden"], inp["top_k_index"], inp["top_k_weights"], gu, dn,
+                                 out_dtype=torch.float32, **kw)
+    out16 = m.moeq_experts_forward(inp["hidden"], inp["top_k_index"], inp["top_k_weights"], gu, dn,
+                                   out_dtype=torch.bfloat16, **kw)
     torch.cuda.synchronize()
+    assert torch.equal(out16.view(torch.int16), out.to(torch.bfloat16).view(torch.int16))
     return out
 
 
