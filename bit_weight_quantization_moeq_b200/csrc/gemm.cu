@@ -13,11 +13,12 @@
 // Tile = 128 weight rows (UMMA M, operand A) x up to 256 tokens (UMMA N, operand B) x
 // K in steps of 64 (one NF4 block, one 128-byte swizzle row).  Both operands are fp16
 // (weights dequantized to fp16, activations and h stored as fp16), accumulation fp32.
-//   warps 0-3  epilogue: TMEM -> registers (tcgen05.ld), SiLU*up or weighted slot stores
-//   warps 4-7  dequant: packed codes (TMA'd into SMEM) -> fp16 A tile in the UMMA
-//              K-major 128B-swizzled layout, one weight row per thread
-//   warp 8     producer: TMA of the token tile (B, 128B swizzle) and of the code tiles
-//   warp 9     TMEM allocation and the single-thread tcgen05.mma issue
+//   warps 0-3   epilogue: TMEM -> registers (tcgen05.ld), SiLU*up or weighted slot stores
+//   warps 4-11  dequant: packed codes (TMA'd into SMEM) -> fp16 A tile in the UMMA
+//               K-major 128B-swizzled layout, half a weight row per thread per stage
+//               (two warps per SM sub-partition, so one hides the other's latency)
+//   warp 12     producer: TMA of the token tile (B, 128B swizzle) and of the code tiles
+//   warp 13     TMEM allocation and the single-thread tcgen05.mma issue
 // Accumulators are double-buffered in TMEM (2 x 256 fp32 columns) so the epilogue of
 // one tile overlaps the mainloop of the next.  The CTA is persistent over a tile list
 // derived on the device from the routing (per-expert token counts).
@@ -38,7 +39,10 @@ constexpr int BM = 128;
 constexpr int BN = kTileN;  // 256
 constexpr int BK = 64;
 constexpr int kStages = 4;
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
+constexpr int kDequantWarps = 8;
+constexpr int kProducerWarp = 12;
+constexpr int kMmaWarp = 13;
 constexpr int kGroupM = 16;  // m-tiles walked per token tile before moving on (L2 reuse)
 constexpr uint32_t kABytes = BM * BK * 2;
 constexpr uint32_t kBBytes = BN * BK * 2;
@@ -120,6 +124,14 @@ __device__ __forceinline__ void sts_u4(uint32_t addr, uint32_t a, uint32_t b, ui
   asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
 }
+// (a.x * s, a.y * s) with one packed fp32x2 multiply, each product rounded once
+__device__ __forceinline__ float2 fmul2(float2 a, float s) {
+  uint64_t r;
+  const uint64_t x = (static_cast<uint64_t>(__float_as_uint(a.y)) << 32) | __float_as_uint(a.x);
+  const uint64_t y = (static_cast<uint64_t>(__float_as_uint(s)) << 32) | __float_as_uint(s);
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(x), "l"(y));
+  return make_float2(__uint_as_float(static_cast<uint32_t>(r)), __uint_as_float(static_cast<uint32_t>(r >> 32)));
+}
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t *>(&h);
@@ -160,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(BAR(s), 1);           // tma_full: producer arrive + tx bytes
-      mbar_init(BAR(4 + s), 4);       // a_full: one arrival per dequant warp
+      mbar_init(BAR(4 + s), kDequantWarps);  // a_full: one arrival per dequant warp
       mbar_init(BAR(8 + s), 1);       // empty: MMA commit
     }
     for (int b = 0; b < 2; ++b) {
@@ -184,11 +196,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       *reinterpret_cast<float *>(smem + kStages * CF::kStageBytes + code * 256 + l * 4) = cv[code];
     }
   }
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     for (int i = 0; i < 5; ++i) tma_prefetch_desc(&maps.b[i]);
     tma_prefetch_desc(&maps.codes);
   }
@@ -200,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total_tiles = args.ntp[args.E] * args.MT;
   const int nk = args.nk;
 
-  if (warp == 8) {
+  if (warp == kProducerWarp) {
     // ---------------- producer ----------------
     if (lane == 0) {
       uint32_t it = 0;
@@ -237,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       uint32_t it = 0, acc_it = 0;
@@ -281,7 +293,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ---------------- dequant ----------------
-    const int r = threadIdx.x - 128;  // tile row = TMEM lane = A row
+    const int dt = threadIdx.x - 128;
+    const int r = dt & 127;           // tile row = TMEM lane = A row (a warp: 32 consecutive rows)
+    const int half = dt >> 7;         // which 32 of the stage's 64 K elements
     const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
     uint32_t it = 0;
     bool ok = true;
@@ -307,13 +321,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (MODE != MOEQ_INT8_ROW && kb + 2 < nk) a_nn = load_absmax<MODE>(args, t.e, wr, kb + 2);
         if (!mbar_wait(BAR(s), ph, abort_flag, args.status)) { ok = false; break; }
         const uint32_t st = sbase + s * CF::kStageBytes;
-        const uint32_t crow = st + kABytes + kBBytes + cr * CF::kCodeRow;
+        const uint32_t crow = st + kABytes + kBBytes + cr * CF::kCodeRow + half * (CF::kCodeRow / 2);
         const uint32_t arow = st + r * 128;
         const uint32_t sw = static_cast<uint32_t>(r & 7);
         if (MODE == MOEQ_INT8_ROW) {
+          // 32 int8 codes -> 32 fp16 values (exact), chunks 4*half .. 4*half+3
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const uint4 cw = lds_u4(crow + q4 * 16);
+          for (int q2 = 0; q2 < 2; ++q2) {
+            const uint4 cw = lds_u4(crow + q2 * 16);
             const uint32_t wv[4] = {cw.x, cw.y, cw.z, cw.w};
             uint32_t o[8];
 #pragma unroll
@@ -326,27 +341,29 @@ __global__ void __launch_bounds__(kThreads, 1)
               o[2 * wi] = pack_f16(f[0], f[1]);
               o[2 * wi + 1] = pack_f16(f[2], f[3]);
             }
-            // 16 elements = two 16-byte chunks (2*q4, 2*q4+1)
-            sts_u4(arow + ((((2 * q4) ^ sw)) << 4), o[0], o[1], o[2], o[3]);
-            sts_u4(arow + ((((2 * q4 + 1) ^ sw)) << 4), o[4], o[5], o[6], o[7]);
+            const uint32_t c0 = static_cast<uint32_t>(4 * half + 2 * q2);
+            sts_u4(arow + ((c0 ^ sw) << 4), o[0], o[1], o[2], o[3]);
+            sts_u4(arow + (((c0 + 1) ^ sw) << 4), o[4], o[5], o[6], o[7]);
           }
         } else {
           const float a = a_cur;
-          const uint4 c0 = lds_u4(crow), c1 = lds_u4(crow + 16);
-          const uint32_t wv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          const uint4 c0 = lds_u4(crow);
+          const uint32_t wv[4] = {c0.x, c0.y, c0.z, c0.w};
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
+          for (int j = 0; j < 4; ++j) {
             const uint32_t hi = (wv[j] >> 4) & 0x0F0F0F0Fu;  // even elements
             const uint32_t lo = wv[j] & 0x0F0F0F0Fu;         // odd elements
             uint32_t o[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const uint32_t sel = 0x5504u | (static_cast<uint32_t>(k) << 4);
-              const float ce = __uint_as_float(lds_u32(lut + __byte_perm(hi, lane4, sel)));
-              const float co = __uint_as_float(lds_u32(lut + __byte_perm(lo, lane4, sel)));
-              o[k] = pack_f16(__fmul_rn(ce, a), __fmul_rn(co, a));
+              float2 c;
+              c.x = __uint_as_float(lds_u32(lut + __byte_perm(hi, lane4, sel)));
+              c.y = __uint_as_float(lds_u32(lut + __byte_perm(lo, lane4, sel)));
+              const float2 w = fmul2(c, a);
+              o[k] = pack_f16(w.x, w.y);
             }
-            sts_u4(arow + ((static_cast<uint32_t>(j) ^ sw) << 4), o[0], o[1], o[2], o[3]);
+            sts_u4(arow + ((static_cast<uint32_t>(4 * half + j) ^ sw) << 4), o[0], o[1], o[2], o[3]);
           }
           a_cur = a_nxt;
           a_nxt = a_nn;
@@ -385,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float g = sgate ? rcv : own;
             const float u = sgate ? own : rcv;
             const int col = c * 32 + (sgate ? 16 : 0) + q;
-            float hval = g / (1.0f + __expf(-g)) * u;
+            float hval = __fdividef(g, 1.0f + __expf(-g)) * u;
             if (col < t.count) {
               if (fabsf(hval) > 65504.0f) {
                 report(args.status, MOEQ_ERR_RANGE);
@@ -431,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }

@@ -73,6 +73,24 @@ __device__ __forceinline__ float div_by(float x, float a, float r) {
   return __fmaf_rn(e, r, q0);
 }
 
+// Packed fp32x2 arithmetic: each lane of the pair is one IEEE round-to-nearest
+// operation, exactly as the scalar form.
+__device__ __forceinline__ uint64_t f2u(float lo, float hi) {
+  return (static_cast<uint64_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ float lo_f(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float hi_f(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+
 __device__ __forceinline__ uint4 ld_stream_u4(const void *p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -117,12 +135,21 @@ __device__ __forceinline__ void nf4_quarter(const uint4 v0, const uint4 v1, size
   const float a = m;
   uint32_t code[16];
   if (a == 0.0f || a >= 0x1p-120f) {
+    // the division and the cell map two elements at a time (fp32x2)
     const float r = (a == 0.0f) ? 0.0f : __frcp_rn(a);
+    const uint64_t r2 = f2u(r, r), na2 = f2u(-a, -a);
+    const uint64_t k15 = f2u(15.0f, 15.0f), kc = f2u(12582927.0f, 12582927.0f);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float n = div_by(x[i], a, r);
-      const int c = nf4_cell(n);
-      code[i] = static_cast<uint32_t>(base[c] + (n > thr[c] ? 1 : 0));
+    for (int i = 0; i < 16; i += 2) {
+      const uint64_t x2 = f2u(x[i], x[i + 1]);
+      const uint64_t q0 = mul2(x2, r2);
+      const uint64_t e = fma2(na2, q0, x2);
+      const uint64_t n2 = fma2(e, r2, q0);
+      const uint64_t f2 = fma2(n2, k15, kc);
+      const int c0 = static_cast<int>(static_cast<uint32_t>(f2) & 31u);
+      const int c1 = static_cast<int>(static_cast<uint32_t>(f2 >> 32) & 31u);
+      code[i] = static_cast<uint32_t>(base[c0] + (lo_f(n2) > thr[c0] ? 1 : 0));
+      code[i + 1] = static_cast<uint32_t>(base[c1] + (hi_f(n2) > thr[c1] ? 1 : 0));
     }
   } else {  // tiny (subnormal-range) absmax: plain IEEE divide
 #pragma unroll
@@ -285,12 +312,28 @@ __global__ void k_quant_int8_row(const uint4 *__restrict__ w, uint2 *__restrict_
       float f[8];
       unpack_bf16x8(v[i], f);
       uint32_t b[8];
+      if (fast) {
+        const uint64_t r2 = f2u(r, r), na2 = f2u(-a, -a), k127 = f2u(127.0f, 127.0f);
+        const uint64_t kr = f2u(12582912.0f, 12582912.0f);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float p = __fmul_rn(127.0f, f[j]);  // exact for a bf16 input
-        const float n = fast ? div_by(p, a, r) : __fdiv_rn(p, a);
-        // rint (half to even) by the 1.5*2^23 shift; |n| <= 127 keeps this exact
-        b[j] = static_cast<uint32_t>(__float_as_int(__fadd_rn(n, 12582912.0f))) & 0xffu;
+        for (int j = 0; j < 8; j += 2) {
+          const uint64_t p2 = mul2(k127, f2u(f[j], f[j + 1]));  // 127 x, exact for bf16 x
+          const uint64_t q0 = mul2(p2, r2);
+          const uint64_t e = fma2(na2, q0, p2);
+          const uint64_t n2 = fma2(e, r2, q0);                  // fl(127 x / absmax)
+          // rint (half to even) by adding 1.5*2^23; |n| <= 127 keeps this exact
+          uint64_t one = f2u(1.0f, 1.0f);
+          const uint64_t rr = fma2(n2, one, kr);
+          b[j] = static_cast<uint32_t>(rr) & 0xffu;
+          b[j + 1] = static_cast<uint32_t>(rr >> 32) & 0xffu;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float p = __fmul_rn(127.0f, f[j]);
+          const float n = __fdiv_rn(p, a);
+          b[j] = static_cast<uint32_t>(__float_as_int(__fadd_rn(n, 12582912.0f))) & 0xffu;
+        }
       }
       uint2 o;
       o.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
