@@ -47,6 +47,7 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-load", action="store_true", help="skip the multi-layer quantize-on-load leg")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
     return p.parse_args()
 
@@ -103,6 +104,38 @@ class ClockSampler:
         loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
         return {"sm_mhz": statistics.median(loaded) if loaded else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# cross-rank helpers (host logic; tested with gloo on CPU)
+# ---------------------------------------------------------------------------
+def max_over_ranks(values, device="cpu"):
+    """Element-wise max of a list of floats over all ranks (identity when not distributed)."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if torch.distributed.is_available() and torch.distributed.is_initialized() \
+            and torch.distributed.get_world_size() > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def sum_over_ranks(values, device="cpu"):
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if torch.distributed.is_available() and torch.distributed.is_initialized() \
+            and torch.distributed.get_world_size() > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return t.tolist()
+
+
+def shard_range(n: int, rank: int, world: int):
+    """Contiguous share of n independent units (layers) for `rank`: sizes differ by at most 1."""
+    base, extra = divmod(n, world)
+    start = rank * base + min(rank, extra)
+    return range(start, start + base + (1 if rank < extra else 0))
+
+
+def aggregate_rate(units_per_rank, max_seconds: float) -> float:
+    """Whole-job rate: all ranks' units over the slowest rank's time."""
+    return float(sum(units_per_rank)) / max_seconds
 
 
 # ---------------------------------------------------------------------------
@@ -233,11 +266,9 @@ def run_ours(args, wl, rank, world, dev):
         "gemm_down": sum(el(t[3], t[4]) for t in tevs),
         "combine": sum(el(t[4], t[5]) for t in tevs),
     }
-    vals = torch.tensor([total_ms] + list(comp.values()), dtype=torch.float64, device=f"cuda:{dev}")
-    if world > 1:
-        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
+    vals = max_over_ranks([total_ms] + list(comp.values()), device=f"cuda:{dev}")
     total_ms = float(vals[0])
-    comp = {k: float(v) / args.steps for k, v in zip(comp.keys(), vals[1:].tolist())}
+    comp = {k: float(v) / args.steps for k, v in zip(comp.keys(), vals[1:])}
 
     from bit_weight_quantization_moeq_b200.synth import forward_flops, quantize_bytes
     S = T * K
@@ -246,7 +277,7 @@ def run_ours(args, wl, rank, world, dev):
     n_elem = E * 3 * I * H
     packed_bytes = gu_p.nbytes() + dn_p.nbytes()
     dq_bytes = packed_bytes + 2 * n_elem
-    fwd_tflops = world * flops / (comp["forward"] * 1e-3) / 1e12
+    fwd_tflops = aggregate_rate([flops] * world, comp["forward"] * 1e-3) / 1e12
     # distinct experts hit (for the forward's algorithmic bytes)
     hit = torch.unique(inputs["top_k_index"]).numel()
     fwd_bytes = packed_bytes * hit / E + 2 * T * H * 2 + S * 8
@@ -303,7 +334,50 @@ def run_ours(args, wl, rank, world, dev):
     return result, inputs
 
 
-def run_e2e(wl, dev, steps=3, warmup=1):
+def run_load(wl, rank, world, dev, layers: int):
+    """Quantize-on-load of `layers` layers (sharded over the ranks): each layer's bf16
+    gate_up and down are drawn into one reused staging buffer (not timed), quantized
+    (timed with CUDA events), and the packed layers are kept, as a loader would."""
+    import bit_weight_quantization_moeq_b200 as M
+    from bit_weight_quantization_moeq_b200 import synth
+    d = f"cuda:{dev}"
+    E, H, I, mode = wl.E, wl.H, wl.I, wl.mode
+    mine = shard_range(layers, rank, world)
+    stage_gu = torch.empty((E, 2 * I, H), dtype=torch.bfloat16, device=d)
+    stage_dn = torch.empty((E, H, I), dtype=torch.bfloat16, device=d)
+    qws = torch.empty(max(M.moeq_quantize_workspace(mode, E, 2 * I, H), 16), dtype=torch.uint8, device=d)
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats(d)
+    kept, ms = [], 0.0
+    for layer in mine:
+        s = 100000 + 10 * layer
+        synth.expert_weights(E, 2 * I, H, s, wl.outliers, d, out=stage_gu)
+        synth.expert_weights(E, H, I, s + 1, wl.outliers, d, out=stage_dn)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        if mode == 2:
+            pg, pd = M.moeq_quantize_int8_rowwise(stage_gu), M.moeq_quantize_int8_rowwise(stage_dn)
+        else:
+            pg = M.moeq_quantize_nf4(stage_gu, double_quant=(mode == 1), ws=qws)
+            pd = M.moeq_quantize_nf4(stage_dn, double_quant=(mode == 1), ws=qws)
+        b.record()
+        torch.cuda.synchronize()
+        ms += a.elapsed_time(b)
+        kept.append((pg, pd))
+    peak = torch.cuda.max_memory_allocated(d)
+    packed = sum(p.nbytes() + q.nbytes() for p, q in kept)
+    from bit_weight_quantization_moeq_b200.synth import quantize_bytes
+    per_layer = quantize_bytes(mode, E, 2 * I, H) + quantize_bytes(mode, E, H, I)
+    max_ms = max_over_ranks([ms], device=d)[0]
+    gbs = aggregate_rate([per_layer * len(shard_range(layers, r, world)) for r in range(world)],
+                         max_ms * 1e-3) / 1e9
+    return {"layers": layers, "gbs": round(gbs, 1), "ms_total_max_rank": round(max_ms, 3),
+            "ms_per_layer": round(ms / max(1, len(mine)), 4),
+            "peak_mem_gib_rank0": round(peak / 2**30, 3), "packed_gib_rank0": round(packed / 2**30, 3),
+            "staging": "one reused bf16 layer (gate_up + down), drawn untimed"}
+
+
+def run_e2e(wl, dev, world=1, steps=3, warmup=1):
     """Same forward metric through the C ABI with host buffers: every step copies its
     inputs (bf16 weights, hidden, routing) from pinned host memory, quantizes,
     dequantizes, runs the forward and reads the output back."""
@@ -348,12 +422,12 @@ def run_e2e(wl, dev, steps=3, warmup=1):
         step()
     b.record()
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / steps
+    ms = max_over_ranks([a.elapsed_time(b) / steps], device=d)[0]
     from bit_weight_quantization_moeq_b200.synth import forward_flops
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    return {"value": round(forward_flops(T, K, H, I) / (ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
-            "ms_per_step": round(ms, 3), "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(out_h.numel() * out_h.element_size()),
+    return {"value": round(aggregate_rate([forward_flops(T, K, H, I)] * world, ms * 1e-3) / 1e12, 4),
+            "unit": "TFLOP/s", "ms_per_step": round(ms, 3), "h2d_bytes_per_step": int(h2d) * world,
+            "d2h_bytes_per_step": int(out_h.numel() * out_h.element_size()) * world,
             "note": "step includes the H2D upload of the bf16 weights being quantized on load"}, host
 
 
@@ -397,11 +471,16 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=torch.device(f"cuda:{local}"))
     result, inputs = run_ours(args, wl, rank, world, local)
-    if rank == 0 and world == 1 and not args.no_e2e:
+    if wl.layers > 1 and not args.no_load:
         del inputs
         torch.cuda.empty_cache()
-        result["e2e"], host = run_e2e(wl, local)
-        if not args.no_cpu_baseline:
+        inputs = None
+        result["load"] = run_load(wl, rank, world, local, wl.layers)
+    if not args.no_e2e:
+        del inputs
+        torch.cuda.empty_cache()
+        result["e2e"], host = run_e2e(wl, local, world)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
             tf, tps, qg, desc, thr = oracle_sample(wl, host, args.cpu_seconds)
             result["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                                       "sample": desc, "tokens_per_s": round(tps, 3), "quantize_gbs": round(qg, 4)}
