@@ -24,6 +24,7 @@ SOURCES = {
     "quant.cu": ["-fmad=false"],
     "route.cu": [],
     "gemm.cu": [],
+    "noalloc.cu": [],
 }
 COMMON = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -166,6 +166,22 @@ moeq_status moeq_route(const void *top_k_index, int index_dtype, int T, int K, i
                        int32_t *counts, int32_t *offsets, int32_t *perm, void *ws,
                        size_t ws_bytes, int32_t *d_status, moeq_stream_t stream);
 
+/* The routing step of moeq_route without a workspace, for callers that cannot allocate
+ * device memory: a host runtime that keeps the whole device for its own memory pool and
+ * forbids allocations outside it, or a latency-critical loop in which cudaMalloc/cudaFree
+ * would synchronise the device.  (The pages have no counterpart: this is a library
+ * convenience, not part of the method.)  Same arguments and results as moeq_route, minus
+ * ws/ws_bytes.  Its scratch is a fixed 2 MiB __device__ array inside the library, held by
+ * every GPU that loads the library until the process exits; it covers
+ * 2*ceil(T*K/512)*E*4 + (E+1)*4 bytes (each part rounded up to 256) and larger problems
+ * return MOEQ_ERR_WORKSPACE.  The first call on a device looks up the array's device
+ * address with that device current: make that first call before any stream capture.
+ * All calls share the array; calls that overlap on the GPU (e.g. on two unordered
+ * streams) race on it.  Allocates nothing, frees nothing. */
+moeq_status moeq_route_noalloc(const void *top_k_index, int index_dtype, int T, int K, int E,
+                               int32_t *counts, int32_t *offsets, int32_t *perm,
+                               int32_t *d_status, moeq_stream_t stream);
+
 /* Device workspace bytes moeq_route needs.  Host only. */
 size_t moeq_route_workspace(int T, int K, int E);
 
