@@ -53,24 +53,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// As above, but the thread may be suspended in hardware for up to `hint_ns` while the
+// phase is incomplete, instead of returning at once: a waiting warp then takes no issue
+// slots from the warps doing work on the same SM sub-partition.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 
-// Bounded wait: gives up after `limit_ns` of wall time (or when another role has
+// Bounded wait: gives up after kWaitLimitNs of wall time (or when another role has
 // already given up), raises the CTA-wide abort flag and reports MOEQ_ERR_TIMEOUT.
 // Returns false on give-up; the caller then leaves its loop.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legal wait
+constexpr uint32_t kSuspendHintNs = 1000000u;     // each try sleeps at most 1 ms
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                           int32_t *status) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
-        *abort_flag = 1;
-        report(status, MOEQ_ERR_TIMEOUT);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      report(status, MOEQ_ERR_TIMEOUT);
+      return false;
     }
   }
 }

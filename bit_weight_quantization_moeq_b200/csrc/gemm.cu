@@ -13,12 +13,13 @@
 // Tile = 128 weight rows (UMMA M, operand A) x up to 256 tokens (UMMA N, operand B) x
 // K in steps of 64 (one NF4 block, one 128-byte swizzle row).  Both operands are fp16
 // (weights dequantized to fp16, activations and h stored as fp16), accumulation fp32.
-//   warps 0-3   epilogue: TMEM -> registers (tcgen05.ld), SiLU*up or weighted slot stores
-//   warps 4-11  dequant: packed codes (TMA'd into SMEM) -> fp16 A tile in the UMMA
-//               K-major 128B-swizzled layout, half a weight row per thread per stage
-//               (two warps per SM sub-partition, so one hides the other's latency)
-//   warp 12     producer: TMA of the token tile (B, 128B swizzle) and of the code tiles
-//   warp 13     TMEM allocation and the single-thread tcgen05.mma issue
+//   warps 0-7   epilogue: TMEM -> registers (tcgen05.ld), SiLU*up or weighted slot stores;
+//               warp w reads TMEM lanes 32*(w%4).. and half the tile's columns
+//   warps 8-23  dequant: packed codes (TMA'd into SMEM) -> fp16 A tile in the UMMA
+//               K-major 128B-swizzled layout, a quarter of a weight row per thread per
+//               stage (four warps per SM sub-partition hide each other's latency)
+//   warp 24     producer: TMA of the token tile (B, 128B swizzle) and of the code tiles
+//   warp 25     TMEM allocation and the single-thread tcgen05.mma issue
 // Accumulators are double-buffered in TMEM (2 x 256 fp32 columns) so the epilogue of
 // one tile overlaps the mainloop of the next.  The CTA is persistent over a tile list
 // derived on the device from the routing (per-expert token counts).
@@ -38,11 +39,17 @@ namespace moeq {
 constexpr int BM = 128;
 constexpr int BN = kTileN;  // 256
 constexpr int BK = 64;
-constexpr int kStages = 4;
-constexpr int kThreads = 448;
-constexpr int kDequantWarps = 8;
-constexpr int kProducerWarp = 12;
-constexpr int kMmaWarp = 13;
+constexpr int kBStages = 4;          // token tiles (TMA), freed by the MMA
+constexpr int kAStages = 4;          // dequantized weight tiles, freed by the MMA
+constexpr int kEpiWarps = 8;
+constexpr int kDequantGroups = 2;    // groups take alternate K stages
+constexpr int kGroupWarps = 8;       // per group: 128 rows x 2 halves
+constexpr int kDequantWarps = kDequantGroups * kGroupWarps;
+constexpr int kDequantThread0 = kEpiWarps * 32;
+constexpr int kCodeProducerWarp = kEpiWarps + kDequantWarps;
+constexpr int kBProducerWarp = kCodeProducerWarp + 1;
+constexpr int kMmaWarp = kBProducerWarp + 1;
+constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr int kGroupM = 16;  // m-tiles walked per token tile before moving on (L2 reuse)
 constexpr uint32_t kABytes = BM * BK * 2;
 constexpr uint32_t kBBytes = BN * BK * 2;
@@ -52,10 +59,23 @@ template <int MODE>
 struct Cfg {
   static constexpr uint32_t kCodeRow = (MODE == MOEQ_INT8_ROW) ? 64 : 32;  // bytes/row/stage
   static constexpr uint32_t kCodeBytes = BM * kCodeRow;
-  static constexpr uint32_t kStageBytes = kABytes + kBBytes + kCodeBytes;
+  static constexpr int kCStages = (MODE == MOEQ_INT8_ROW) ? 4 : 6;  // packed-code tiles, deep
+  static constexpr uint32_t kBOff = 0;
+  static constexpr uint32_t kAOff = kBOff + kBStages * kBBytes;
+  static constexpr uint32_t kCOff = kAOff + kAStages * kABytes;
+  static constexpr uint32_t kLutOff = kCOff + kCStages * kCodeBytes;
   static constexpr uint32_t kLut = (MODE == MOEQ_INT8_ROW) ? 0 : kLutBytes;
-  static constexpr uint32_t kSmem = kStages * kStageBytes + kLut + 256 + 1024;
+  static constexpr uint32_t kCtrlOff = kLutOff + kLut;
+  static constexpr int kNumBars = 2 * kBStages + 2 * kAStages + 2 * kCStages + 5;
+  static constexpr uint32_t kSmem = kCtrlOff + kNumBars * 8 + 16 + 1024;
 };
+
+// The 16 NormalFloat-4 levels (fp32), the table the packed codes index.
+__constant__ float kNF4Levels[16] = {
+    -1.0f, -0.6961928009986877f, -0.5250730514526367f, -0.39491748809814453f,
+    -0.28444138169288635f, -0.18477343022823334f, -0.09105003625154495f, 0.0f,
+    0.07958029955625534f, 0.16093020141124725f, 0.24611230194568634f, 0.33791524171829224f,
+    0.44070982933044434f, 0.5626170039176941f, 0.7229568362236023f, 1.0f};
 
 struct TmapSet {
   CUtensorMap b[5];  // activation rows, boxes of 16, 32, 64, 128, 256 rows x 64 elements
@@ -108,21 +128,16 @@ __device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a) {
   return t;
 }
 
-__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
+// Shared-memory accesses as plain loads/stores through the dynamic shared buffer, so the
+// compiler is free to interleave the many independent table lookups of a dequant thread.
+__device__ __forceinline__ uint32_t lds_u32(const uint8_t *smem, uint32_t off) {
+  return *reinterpret_cast<const uint32_t *>(smem + off);
 }
-__device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
-  return v;
+__device__ __forceinline__ uint4 lds_u4(const uint8_t *smem, uint32_t off) {
+  return *reinterpret_cast<const uint4 *>(smem + off);
 }
-__device__ __forceinline__ void sts_u4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-               : "memory");
+__device__ __forceinline__ void sts_u4(uint8_t *smem, uint32_t off, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  *reinterpret_cast<uint4 *>(smem + off) = make_uint4(a, b, c, d);
 }
 // (a.x * s, a.y * s) with one packed fp32x2 multiply, each product rounded once
 __device__ __forceinline__ float2 fmul2(float2 a, float s) {
@@ -155,31 +170,48 @@ template <int MODE, int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     k_moe_gemm(const __grid_constant__ TmapSet maps, const GemmArgs args) {
   using CF = Cfg<MODE>;
+  constexpr int kCS = CF::kCStages;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, kept as shared-array arithmetic so accesses stay shared loads
+  uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t lut = sbase + kStages * CF::kStageBytes;
-  uint8_t *ctrl = smem + kStages * CF::kStageBytes + CF::kLut;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl);
-  // bars: [0,4) tma_full, [4,8) a_full, [8,12) empty, [12,14) acc_full, [14,16) acc_empty, 16 drain
-  const uint32_t bar0 = smem_u32(bars);
-  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * i; };
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ctrl + 17 * 8);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 17 * 8 + 4);
+  uint8_t *ctrl = smem + CF::kCtrlOff;
+  const uint32_t bar0 = smem_u32(ctrl);
+  // barriers: token ring full/empty, A ring full/empty, code ring full/empty,
+  // accumulator full/empty (x2), drain
+  auto B_FULL = [&](int i) -> uint32_t { return bar0 + 8u * i; };
+  auto B_EMPTY = [&](int i) -> uint32_t { return bar0 + 8u * (kBStages + i); };
+  auto A_FULL = [&](int i) -> uint32_t { return bar0 + 8u * (2 * kBStages + i); };
+  auto A_EMPTY = [&](int i) -> uint32_t { return bar0 + 8u * (2 * kBStages + kAStages + i); };
+  auto C_FULL = [&](int i) -> uint32_t { return bar0 + 8u * (2 * kBStages + 2 * kAStages + i); };
+  auto C_EMPTY = [&](int i) -> uint32_t { return bar0 + 8u * (2 * kBStages + 2 * kAStages + kCS + i); };
+  constexpr int kAcc0 = 2 * kBStages + 2 * kAStages + 2 * kCS;
+  auto ACC_FULL = [&](int b) -> uint32_t { return bar0 + 8u * (kAcc0 + b); };
+  auto ACC_EMPTY = [&](int b) -> uint32_t { return bar0 + 8u * (kAcc0 + 2 + b); };
+  const uint32_t DRAIN = bar0 + 8u * (kAcc0 + 4);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ctrl + CF::kNumBars * 8);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + CF::kNumBars * 8 + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(BAR(s), 1);           // tma_full: producer arrive + tx bytes
-      mbar_init(BAR(4 + s), kDequantWarps);  // a_full: one arrival per dequant warp
-      mbar_init(BAR(8 + s), 1);       // empty: MMA commit
+    for (int i = 0; i < kBStages; ++i) {
+      mbar_init(B_FULL(i), 1);        // producer arrive + tx bytes
+      mbar_init(B_EMPTY(i), 1);       // MMA commit
+    }
+    for (int i = 0; i < kAStages; ++i) {
+      mbar_init(A_FULL(i), kGroupWarps);  // one arrival per warp of the dequant group
+      mbar_init(A_EMPTY(i), 1);           // MMA commit
+    }
+    for (int i = 0; i < kCS; ++i) {
+      mbar_init(C_FULL(i), 1);            // producer arrive + tx bytes
+      mbar_init(C_EMPTY(i), kGroupWarps); // the group has read the codes
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(BAR(12 + b), 1);      // acc_full: MMA commit
-      mbar_init(BAR(14 + b), 4);      // acc_empty: one arrival per epilogue warp
+      mbar_init(ACC_FULL(b), 1);          // MMA commit
+      mbar_init(ACC_EMPTY(b), kEpiWarps); // one arrival per epilogue warp
     }
-    mbar_init(BAR(16), 1);            // drain
+    mbar_init(DRAIN, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -188,22 +220,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // that each lane reads its own bank whatever code it looks up.
     for (int i = threadIdx.x; i < 16 * 32; i += kThreads) {
       const int code = i >> 5, l = i & 31;
-      const float cv[16] = {-1.0f, -0.6961928009986877f, -0.5250730514526367f, -0.39491748809814453f,
-                            -0.28444138169288635f, -0.18477343022823334f, -0.09105003625154495f, 0.0f,
-                            0.07958029955625534f, 0.16093020141124725f, 0.24611230194568634f,
-                            0.33791524171829224f, 0.44070982933044434f, 0.5626170039176941f,
-                            0.7229568362236023f, 1.0f};
-      *reinterpret_cast<float *>(smem + kStages * CF::kStageBytes + code * 256 + l * 4) = cv[code];
+      *reinterpret_cast<float *>(smem + CF::kLutOff + code * 256 + l * 4) = kNF4Levels[code];
     }
   }
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
-  if (warp == kProducerWarp && lane == 0) {
+  if (warp == kBProducerWarp && lane == 0) {
     for (int i = 0; i < 5; ++i) tma_prefetch_desc(&maps.b[i]);
-    tma_prefetch_desc(&maps.codes);
   }
+  if (warp == kCodeProducerWarp && lane == 0) tma_prefetch_desc(&maps.codes);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -212,8 +239,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total_tiles = args.ntp[args.E] * args.MT;
   const int nk = args.nk;
 
-  if (warp == kProducerWarp) {
-    // ---------------- producer ----------------
+  if (warp == kCodeProducerWarp) {
+    // ---------------- packed-code producer ----------------
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
@@ -227,23 +254,46 @@ __global__ void __launch_bounds__(kThreads, 1)
           y0 = t.e * args.R + t.m * 128;
           y1 = y0 + 64;
         }
-        const uint32_t tx = (16u << t.nbox) * 128u + CF::kCodeBytes;
         for (int kb = 0; kb < nk; ++kb, ++it) {
-          const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
-          if (!mbar_wait(BAR(8 + s), ph ^ 1u, abort_flag, args.status)) { ok = false; break; }
-          const uint32_t st = sbase + s * CF::kStageBytes;
-          mbar_arrive_expect_tx(BAR(s), tx);
-          tma_load_2d(st + kABytes, &maps.b[t.nbox], kb * BK, t.row0, BAR(s));
-          tma_load_2d(st + kABytes + kBBytes, &maps.codes, kb * CF::kCodeRow, y0, BAR(s));
-          tma_load_2d(st + kABytes + kBBytes + 64 * CF::kCodeRow, &maps.codes, kb * CF::kCodeRow, y1, BAR(s));
+          const uint32_t s = it % kCS, ph = (it / kCS) & 1u;
+          if (!mbar_wait(C_EMPTY(s), ph ^ 1u, abort_flag, args.status)) { ok = false; break; }
+          const uint32_t dst = sbase + CF::kCOff + s * CF::kCodeBytes;
+          mbar_arrive_expect_tx(C_FULL(s), CF::kCodeBytes);
+          tma_load_2d(dst, &maps.codes, kb * CF::kCodeRow, y0, C_FULL(s));
+          tma_load_2d(dst + 64 * CF::kCodeRow, &maps.codes, kb * CF::kCodeRow, y1, C_FULL(s));
         }
       }
       // drain: every copy issued lands before the CTA may exit
-      const uint32_t n = it < kStages ? it : kStages;
+      const uint32_t n = it < static_cast<uint32_t>(kCS) ? it : static_cast<uint32_t>(kCS);
       for (uint32_t d = 0; d < n; ++d) {
         const uint32_t j = it - 1 - d;
-        uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(BAR(j % kStages), (j / kStages) & 1u)) {
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(C_FULL(j % kCS), (j / kCS) & 1u)) {
+          if (globaltimer() - t0 > kWaitLimitNs) break;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == kBProducerWarp) {
+    // ---------------- token-tile producer ----------------
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        const Tile t = decode_tile(tile, args);
+        const uint32_t tx = (16u << t.nbox) * 128u;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const uint32_t s = it % kBStages, ph = (it / kBStages) & 1u;
+          if (!mbar_wait(B_EMPTY(s), ph ^ 1u, abort_flag, args.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(B_FULL(s), tx);
+          tma_load_2d(sbase + CF::kBOff + s * kBBytes, &maps.b[t.nbox], kb * BK, t.row0, B_FULL(s));
+        }
+      }
+      const uint32_t n = it < static_cast<uint32_t>(kBStages) ? it : static_cast<uint32_t>(kBStages);
+      for (uint32_t d = 0; d < n; ++d) {
+        const uint32_t j = it - 1 - d;
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(B_FULL(j % kBStages), (j / kBStages) & 1u)) {
           if (globaltimer() - t0 > kWaitLimitNs) break;
         }
       }
@@ -257,45 +307,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++acc_it) {
         const Tile t = decode_tile(tile, args);
         const uint32_t b = acc_it & 1u, aph = (acc_it >> 1) & 1u;
-        if (!mbar_wait(BAR(14 + b), aph ^ 1u, abort_flag, args.status)) break;
+        if (!mbar_wait(ACC_EMPTY(b), aph ^ 1u, abort_flag, args.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * 256u;
         const uint32_t n_mma = static_cast<uint32_t>((t.count + 15) & ~15);
         const uint32_t idesc = umma_idesc_f16_m128(n_mma);
         for (int kb = 0; kb < nk; ++kb, ++it) {
-          const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
-          if (!mbar_wait(BAR(s), ph, abort_flag, args.status) ||
-              !mbar_wait(BAR(4 + s), ph, abort_flag, args.status)) {
+          const uint32_t bs = it % kBStages, bph = (it / kBStages) & 1u;
+          const uint32_t as = it % kAStages, aph2 = (it / kAStages) & 1u;
+          if (!mbar_wait(B_FULL(bs), bph, abort_flag, args.status) ||
+              !mbar_wait(A_FULL(as), aph2, abort_flag, args.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t st = sbase + s * CF::kStageBytes;
-          const uint64_t adesc = umma_desc_sw128(st);
-          const uint64_t bdesc = umma_desc_sw128(st + kABytes);
+          const uint64_t adesc = umma_desc_sw128(sbase + CF::kAOff + as * kABytes);
+          const uint64_t bdesc = umma_desc_sw128(sbase + CF::kBOff + bs * kBBytes);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             // +32 bytes along K inside the 128-byte swizzle row = +2 in the start field
             umma_f16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
           }
-          umma_commit(BAR(8 + s));
+          umma_commit(B_EMPTY(bs));
+          umma_commit(A_EMPTY(as));
         }
         if (!ok) break;
-        umma_commit(BAR(12 + b));
+        umma_commit(ACC_FULL(b));
       }
       // drain: all issued MMAs complete before TMEM is freed
-      umma_commit(BAR(16));
-      uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(BAR(16), 0)) {
+      umma_commit(DRAIN);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(DRAIN, 0)) {
         if (globaltimer() - t0 > kWaitLimitNs) break;
       }
     }
     __syncwarp();
-  } else if (warp >= 4) {
-    // ---------------- dequant ----------------
-    const int dt = threadIdx.x - 128;
-    const int r = dt & 127;           // tile row = TMEM lane = A row (a warp: 32 consecutive rows)
-    const int half = dt >> 7;         // which 32 of the stage's 64 K elements
+  } else if (warp >= kEpiWarps) {
+    // ---------------- dequant (two groups, alternate K stages) ----------------
+    const int dt = threadIdx.x - kDequantThread0;
+    const int group = dt / (kGroupWarps * 32);
+    const int gt = dt - group * (kGroupWarps * 32);
+    const int r = gt & 127;            // tile row = TMEM lane = A row (a warp: 32 consecutive rows)
+    const int half = gt >> 7;          // which 32 of the stage's 64 K elements
     const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
     uint32_t it = 0;
     bool ok = true;
@@ -310,25 +363,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         wr = t.m * 128 + r;
         cr = r;
       }
-      float a_cur = 0.f, a_nxt = 0.f;
-      if (MODE != MOEQ_INT8_ROW) {
-        a_cur = load_absmax<MODE>(args, t.e, wr, 0);
-        if (nk > 1) a_nxt = load_absmax<MODE>(args, t.e, wr, 1);
-      }
+      float a_pref = 0.f;
+      bool have_pref = false;
       for (int kb = 0; kb < nk; ++kb, ++it) {
-        const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
-        float a_nn = 0.f;
-        if (MODE != MOEQ_INT8_ROW && kb + 2 < nk) a_nn = load_absmax<MODE>(args, t.e, wr, kb + 2);
-        if (!mbar_wait(BAR(s), ph, abort_flag, args.status)) { ok = false; break; }
-        const uint32_t st = sbase + s * CF::kStageBytes;
-        const uint32_t crow = st + kABytes + kBBytes + cr * CF::kCodeRow + half * (CF::kCodeRow / 2);
-        const uint32_t arow = st + r * 128;
+        if (static_cast<int>(it % kDequantGroups) != group) continue;
+        float a = 0.f;
+        if (MODE != MOEQ_INT8_ROW) {
+          a = have_pref ? a_pref : load_absmax<MODE>(args, t.e, wr, kb);
+          have_pref = kb + kDequantGroups < nk;
+          if (have_pref) a_pref = load_absmax<MODE>(args, t.e, wr, kb + kDequantGroups);
+        }
+        const uint32_t cs = it % kCS, cph = (it / kCS) & 1u;
+        const uint32_t as = it % kAStages, aph = (it / kAStages) & 1u;
+        if (!mbar_wait(C_FULL(cs), cph, abort_flag, args.status)) { ok = false; break; }
+        // this thread's codes: 16 bytes (NF4, 32 nibbles) or 32 bytes (int8) of its row
+        const uint32_t crow = CF::kCOff + cs * CF::kCodeBytes + cr * CF::kCodeRow + half * (CF::kCodeRow / 2);
+        uint4 cw0 = lds_u4(smem, crow), cw1 = make_uint4(0, 0, 0, 0);
+        if (MODE == MOEQ_INT8_ROW) cw1 = lds_u4(smem, crow + 16);
+        if (!mbar_wait(A_EMPTY(as), aph ^ 1u, abort_flag, args.status)) { ok = false; break; }
+        const uint32_t arow = CF::kAOff + as * kABytes + r * 128;
         const uint32_t sw = static_cast<uint32_t>(r & 7);
+        const uint32_t c0 = static_cast<uint32_t>(4 * half);  // first 16-byte chunk of the half row
         if (MODE == MOEQ_INT8_ROW) {
-          // 32 int8 codes -> 32 fp16 values (exact), chunks 4*half .. 4*half+3
+          // 32 int8 codes -> 32 fp16 values (exact)
 #pragma unroll
           for (int q2 = 0; q2 < 2; ++q2) {
-            const uint4 cw = lds_u4(crow + q2 * 16);
+            const uint4 cw = q2 ? cw1 : cw0;
             const uint32_t wv[4] = {cw.x, cw.y, cw.z, cw.w};
             uint32_t o[8];
 #pragma unroll
@@ -341,14 +401,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               o[2 * wi] = pack_f16(f[0], f[1]);
               o[2 * wi + 1] = pack_f16(f[2], f[3]);
             }
-            const uint32_t c0 = static_cast<uint32_t>(4 * half + 2 * q2);
-            sts_u4(arow + ((c0 ^ sw) << 4), o[0], o[1], o[2], o[3]);
-            sts_u4(arow + (((c0 + 1) ^ sw) << 4), o[4], o[5], o[6], o[7]);
+            const uint32_t cq = c0 + 2 * q2;
+            sts_u4(smem, arow + ((cq ^ sw) << 4), o[0], o[1], o[2], o[3]);
+            sts_u4(smem, arow + (((cq + 1) ^ sw) << 4), o[4], o[5], o[6], o[7]);
           }
         } else {
-          const float a = a_cur;
-          const uint4 c0 = lds_u4(crow);
-          const uint32_t wv[4] = {c0.x, c0.y, c0.z, c0.w};
+          const uint32_t wv[4] = {cw0.x, cw0.y, cw0.z, cw0.w};
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const uint32_t hi = (wv[j] >> 4) & 0x0F0F0F0Fu;  // even elements
@@ -358,32 +416,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int k = 0; k < 4; ++k) {
               const uint32_t sel = 0x5504u | (static_cast<uint32_t>(k) << 4);
               float2 c;
-              c.x = __uint_as_float(lds_u32(lut + __byte_perm(hi, lane4, sel)));
-              c.y = __uint_as_float(lds_u32(lut + __byte_perm(lo, lane4, sel)));
+              c.x = __uint_as_float(lds_u32(smem, CF::kLutOff + __byte_perm(hi, lane4, sel)));
+              c.y = __uint_as_float(lds_u32(smem, CF::kLutOff + __byte_perm(lo, lane4, sel)));
               const float2 w = fmul2(c, a);
               o[k] = pack_f16(w.x, w.y);
             }
-            sts_u4(arow + ((static_cast<uint32_t>(4 * half + j) ^ sw) << 4), o[0], o[1], o[2], o[3]);
+            sts_u4(smem, arow + (((c0 + j) ^ sw) << 4), o[0], o[1], o[2], o[3]);
           }
-          a_cur = a_nxt;
-          a_nxt = a_nn;
         }
+        // the proxy fence orders this thread's generic shared-memory accesses (the A
+        // stores, the code loads) before the tensor core's reads and the next TMA write
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(4 + s));
+        if (lane == 0) {
+          mbar_arrive(A_FULL(as));
+          mbar_arrive(C_EMPTY(cs));
+        }
       }
     }
   } else {
-    // ---------------- epilogue (warps 0-3) ----------------
-    const int r = warp * 32 + lane;
+    // ---------------- epilogue (warps 0-7) ----------------
+    const int quad = warp & 3;                 // TMEM lanes 32*quad .. 32*quad+31
+    const int col0 = (warp >> 2) * (BN / 2);   // this warp's half of the tile's columns
+    const int r = quad * 32 + lane;
     uint32_t acc_it = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++acc_it) {
       const Tile t = decode_tile(tile, args);
       const uint32_t b = acc_it & 1u, aph = (acc_it >> 1) & 1u;
-      if (!mbar_wait(BAR(12 + b), aph, abort_flag, args.status)) break;
+      if (!mbar_wait(ACC_FULL(b), aph, abort_flag, args.status)) break;
       tc_fence_after();
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + b * 256u;
-      const int nch = (t.count + 31) >> 5;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + b * 256u;
+      const int ncols = min(BN / 2, t.count - col0);   // may be <= 0: nothing to do
+      const int nch = ncols > 0 ? (ncols + 31) >> 5 : 0;
       if (KIND == 0) {
         const int sgate = lane & 1;
         const int j = t.m * 64 + (r >> 1);
@@ -392,16 +456,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           step = __fdiv_rn(__ldg(args.absmax + static_cast<size_t>(t.e) * args.R + sgate * args.I + j), 127.0f);
         for (int c = 0; c < nch; ++c) {
           uint32_t v[32];
-          tmem_ld_32x32b_x32(tbase + c * 32, v);
+          tmem_ld_32x32b_x32(tbase + col0 + c * 32, v);
           tmem_ld_wait();
 #pragma unroll
           for (int q = 0; q < 16; ++q) {
-            const float own = __uint_as_float(sgate ? v[16 + q] : v[q]) * step;
-            const float snd = __uint_as_float(sgate ? v[q] : v[16 + q]) * step;
+            float own = __uint_as_float(sgate ? v[16 + q] : v[q]);
+            float snd = __uint_as_float(sgate ? v[q] : v[16 + q]);
+            if (MODE == MOEQ_INT8_ROW) {
+              own *= step;
+              snd *= step;
+            }
             const float rcv = __shfl_xor_sync(0xffffffffu, snd, 1);
             const float g = sgate ? rcv : own;
             const float u = sgate ? own : rcv;
-            const int col = c * 32 + (sgate ? 16 : 0) + q;
+            const int col = col0 + c * 32 + (sgate ? 16 : 0) + q;
             float hval = __fdividef(g, 1.0f + __expf(-g)) * u;
             if (col < t.count) {
               if (fabsf(hval) > 65504.0f) {
@@ -419,9 +487,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           step = __fdiv_rn(__ldg(args.absmax + static_cast<size_t>(t.e) * args.R + i), 127.0f);
         for (int c = 0; c < nch; ++c) {
           uint32_t v[32];
-          tmem_ld_32x32b_x32(tbase + c * 32, v);
+          tmem_ld_32x32b_x32(tbase + col0 + c * 32, v);
           tmem_ld_wait();
-          const int colL = c * 32 + lane;
+          const int colL = col0 + c * 32 + lane;
           int p = 0;
           float wv = 0.0f;
           if (colL < t.count) {
@@ -435,14 +503,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int q = 0; q < 32; ++q) {
             const int pq = __shfl_sync(0xffffffffu, p, q);
             const float wq = __shfl_sync(0xffffffffu, wv, q);
-            if (c * 32 + q < t.count)
-              args.slot_out[static_cast<size_t>(pq) * args.R + i] = wq * (__uint_as_float(v[q]) * step);
+            if (col0 + c * 32 + q < t.count)
+              args.slot_out[static_cast<size_t>(pq) * args.R + i] =
+                  MODE == MOEQ_INT8_ROW ? wq * (__uint_as_float(v[q]) * step) : wq * __uint_as_float(v[q]);
           }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(14 + b));
+      if (lane == 0) mbar_arrive(ACC_EMPTY(b));
     }
   }
 
