@@ -10,18 +10,20 @@
 //   down:     slot[p, i] = w_p * (h_s . D_e[i])   with p = perm[s] the (t, k) pair of s
 // over the expert-sorted rows s of each expert e.
 //
-// Tile = 128 weight rows (UMMA M, operand A) x up to 256 tokens (UMMA N, operand B) x
-// K in steps of 64 (one NF4 block, one 128-byte swizzle row).  Both operands are fp16
-// (weights dequantized to fp16, activations and h stored as fp16), accumulation fp32.
+// Tile = 128 weight rows (UMMA M, operand A) x up to 192 tokens (UMMA N, operand B) x
+// K in steps of 64 (one NF4 block).  Both operands are fp16 (weights dequantized to fp16,
+// activations and h stored as fp16), accumulation fp32.  The dequantized weights never
+// touch shared memory: the dequant warps store them straight into tensor memory
+// (tcgen05.st) and the MMA reads operand A from there; only the token tiles (TMA, 128B
+// swizzle) and the packed codes go through shared memory.
 //   warps 0-7   epilogue: TMEM -> registers (tcgen05.ld), SiLU*up or weighted slot stores;
 //               warp w reads TMEM lanes 32*(w%4).. and half the tile's columns
-//   warps 8-23  dequant: packed codes (TMA'd into SMEM) -> fp16 A tile in the UMMA
-//               K-major 128B-swizzled layout, a quarter of a weight row per thread per
-//               stage (four warps per SM sub-partition hide each other's latency)
+//   warps 8-23  dequant: packed codes (TMA'd into SMEM) -> fp16 A stage in TMEM, one
+//               weight row per thread; four groups of 4 warps take K stages in turn
 //   warp 24     producer: TMA of the token tile (B, 128B swizzle) and of the code tiles
 //   warp 25     TMEM allocation and the single-thread tcgen05.mma issue
-// Accumulators are double-buffered in TMEM (2 x 256 fp32 columns) so the epilogue of
-// one tile overlaps the mainloop of the next.  The CTA is persistent over a tile list
+// TMEM (512 columns): two 192-column fp32 accumulators (the epilogue of one tile overlaps
+// the mainloop of the next) and a 4-deep ring of 32-column fp16 A stages.  The CTA is persistent over a tile list
 // derived on the device from the routing (per-expert token counts).
 // Every mbarrier wait is bounded (2 s); a timeout raises MOEQ_ERR_TIMEOUT and the CTA
 // drains its in-flight copies and MMAs, frees TMEM and returns.
@@ -37,13 +39,16 @@
 namespace moeq {
 
 constexpr int BM = 128;
-constexpr int BN = kTileN;  // 256
+constexpr int BN = kTileN;  // 192
 constexpr int BK = 64;
-constexpr int kBStages = 4;          // token tiles (TMA), freed by the MMA
-constexpr int kAStages = 4;          // dequantized weight tiles, freed by the MMA
+constexpr int kBStages = 6;          // token tiles (TMA), freed by the MMA
+constexpr int kAStages = 4;          // dequantized weight stages in TMEM, freed by the MMA
+constexpr uint32_t kAccCols = BN;    // fp32 columns per accumulator
+constexpr uint32_t kACol0 = 2 * kAccCols;  // first TMEM column of the A ring
+constexpr uint32_t kAStageCols = 32;       // 64 fp16 per row = 32 columns
 constexpr int kEpiWarps = 8;
-constexpr int kDequantGroups = 2;    // groups take alternate K stages
-constexpr int kGroupWarps = 8;       // per group: 128 rows x 2 halves
+constexpr int kDequantGroups = 4;    // groups take K stages in turn
+constexpr int kGroupWarps = 4;       // per group: 128 rows, one per thread
 constexpr int kDequantWarps = kDequantGroups * kGroupWarps;
 constexpr int kDequantThread0 = kEpiWarps * 32;
 constexpr int kCodeProducerWarp = kEpiWarps + kDequantWarps;
@@ -51,18 +56,19 @@ constexpr int kBProducerWarp = kCodeProducerWarp + 1;
 constexpr int kMmaWarp = kBProducerWarp + 1;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr int kGroupM = 16;  // m-tiles walked per token tile before moving on (L2 reuse)
-constexpr uint32_t kABytes = BM * BK * 2;
 constexpr uint32_t kBBytes = BN * BK * 2;
-constexpr uint32_t kLutBytes = 16 * 256;
+// NF4 pair table: for every code byte (two 4-bit codes) the two fp32 levels, one copy
+// per lane: entry (byte, lane) at byte*256 + lane*8, so the address is one byte permute
+// and each lane's 8-byte load hits its own banks.
+constexpr uint32_t kLutBytes = 256 * 256;
 
 template <int MODE>
 struct Cfg {
   static constexpr uint32_t kCodeRow = (MODE == MOEQ_INT8_ROW) ? 64 : 32;  // bytes/row/stage
   static constexpr uint32_t kCodeBytes = BM * kCodeRow;
-  static constexpr int kCStages = (MODE == MOEQ_INT8_ROW) ? 4 : 6;  // packed-code tiles, deep
+  static constexpr int kCStages = (MODE == MOEQ_INT8_ROW) ? 8 : 4;  // packed-code tiles
   static constexpr uint32_t kBOff = 0;
-  static constexpr uint32_t kAOff = kBOff + kBStages * kBBytes;
-  static constexpr uint32_t kCOff = kAOff + kAStages * kABytes;
+  static constexpr uint32_t kCOff = kBOff + kBStages * kBBytes;
   static constexpr uint32_t kLutOff = kCOff + kCStages * kCodeBytes;
   static constexpr uint32_t kLut = (MODE == MOEQ_INT8_ROW) ? 0 : kLutBytes;
   static constexpr uint32_t kCtrlOff = kLutOff + kLut;
@@ -77,8 +83,10 @@ __constant__ float kNF4Levels[16] = {
     0.07958029955625534f, 0.16093020141124725f, 0.24611230194568634f, 0.33791524171829224f,
     0.44070982933044434f, 0.5626170039176941f, 0.7229568362236023f, 1.0f};
 
+__device__ __forceinline__ uint32_t box_rows(int nbox) { return nbox < 4 ? (16u << nbox) : 192u; }
+
 struct TmapSet {
-  CUtensorMap b[5];  // activation rows, boxes of 16, 32, 64, 128, 256 rows x 64 elements
+  CUtensorMap b[5];  // activation rows, boxes of 16, 32, 64, 128, 192 rows x 64 elements
   CUtensorMap codes; // packed codes, [E*R rows, bytes per row], box 64 rows x kCodeRow
 };
 
@@ -136,9 +144,7 @@ __device__ __forceinline__ uint32_t lds_u32(const uint8_t *smem, uint32_t off) {
 __device__ __forceinline__ uint4 lds_u4(const uint8_t *smem, uint32_t off) {
   return *reinterpret_cast<const uint4 *>(smem + off);
 }
-__device__ __forceinline__ void sts_u4(uint8_t *smem, uint32_t off, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  *reinterpret_cast<uint4 *>(smem + off) = make_uint4(a, b, c, d);
-}
+
 // (a.x * s, a.y * s) with one packed fp32x2 multiply, each product rounded once
 __device__ __forceinline__ float2 fmul2(float2 a, float s) {
   uint64_t r;
@@ -216,11 +222,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_fence_init();
   }
   if (MODE != MOEQ_INT8_ROW) {
-    // NF4 level table, one copy per lane: entry (code, lane) at code*256 + lane*4, so
-    // that each lane reads its own bank whatever code it looks up.
-    for (int i = threadIdx.x; i < 16 * 32; i += kThreads) {
-      const int code = i >> 5, l = i & 31;
-      *reinterpret_cast<float *>(smem + CF::kLutOff + code * 256 + l * 4) = kNF4Levels[code];
+    // NF4 pair table (see kLutBytes): entry (byte, lane) = (c[byte >> 4], c[byte & 15])
+    for (int i = threadIdx.x; i < 256 * 32; i += kThreads) {
+      const int byte = i >> 5, l = i & 31;
+      *reinterpret_cast<float2 *>(smem + CF::kLutOff + byte * 256 + l * 8) =
+          make_float2(kNF4Levels[byte >> 4], kNF4Levels[byte & 15]);
     }
   }
   if (warp == kMmaWarp) {
@@ -281,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
         const Tile t = decode_tile(tile, args);
-        const uint32_t tx = (16u << t.nbox) * 128u;
+        const uint32_t tx = box_rows(t.nbox) * 128u;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % kBStages, ph = (it / kBStages) & 1u;
           if (!mbar_wait(B_EMPTY(s), ph ^ 1u, abort_flag, args.status)) { ok = false; break; }
@@ -309,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t b = acc_it & 1u, aph = (acc_it >> 1) & 1u;
         if (!mbar_wait(ACC_EMPTY(b), aph ^ 1u, abort_flag, args.status)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + b * 256u;
+        const uint32_t d_tmem = tmem_base + b * kAccCols;
         const uint32_t n_mma = static_cast<uint32_t>((t.count + 15) & ~15);
         const uint32_t idesc = umma_idesc_f16_m128(n_mma);
         for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -321,12 +327,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t adesc = umma_desc_sw128(sbase + CF::kAOff + as * kABytes);
+          const uint32_t a_tmem = tmem_base + kACol0 + as * kAStageCols;
           const uint64_t bdesc = umma_desc_sw128(sbase + CF::kBOff + bs * kBBytes);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            // +32 bytes along K inside the 128-byte swizzle row = +2 in the start field
-            umma_f16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
+            // K = 16 per MMA: +8 TMEM columns of A, +32 bytes (+2 in the start field) of B
+            umma_f16_ts(d_tmem, a_tmem + 8u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
           }
           umma_commit(B_EMPTY(bs));
           umma_commit(A_EMPTY(as));
@@ -343,13 +349,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= kEpiWarps) {
-    // ---------------- dequant (two groups, alternate K stages) ----------------
+    // ---------------- dequant (four groups, K stages in turn) ----------------
     const int dt = threadIdx.x - kDequantThread0;
     const int group = dt / (kGroupWarps * 32);
-    const int gt = dt - group * (kGroupWarps * 32);
-    const int r = gt & 127;            // tile row = TMEM lane = A row (a warp: 32 consecutive rows)
-    const int half = gt >> 7;          // which 32 of the stage's 64 K elements
-    const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
+    const int r = dt - group * (kGroupWarps * 32);  // tile row = TMEM lane (warp%4 quadrant)
+    const uint32_t lane8 = static_cast<uint32_t>(lane) * 8u;
+    const uint32_t trow = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kACol0;
     uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
@@ -376,56 +381,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t cs = it % kCS, cph = (it / kCS) & 1u;
         const uint32_t as = it % kAStages, aph = (it / kAStages) & 1u;
         if (!mbar_wait(C_FULL(cs), cph, abort_flag, args.status)) { ok = false; break; }
-        // this thread's codes: 16 bytes (NF4, 32 nibbles) or 32 bytes (int8) of its row
-        const uint32_t crow = CF::kCOff + cs * CF::kCodeBytes + cr * CF::kCodeRow + half * (CF::kCodeRow / 2);
-        uint4 cw0 = lds_u4(smem, crow), cw1 = make_uint4(0, 0, 0, 0);
-        if (MODE == MOEQ_INT8_ROW) cw1 = lds_u4(smem, crow + 16);
+        // this thread's codes: its row of the stage, 32 bytes (NF4) or 64 bytes (int8)
+        const uint32_t crow = CF::kCOff + cs * CF::kCodeBytes + cr * CF::kCodeRow;
+        uint4 cw[CF::kCodeRow / 16];
+#pragma unroll
+        for (int i = 0; i < static_cast<int>(CF::kCodeRow / 16); ++i) cw[i] = lds_u4(smem, crow + 16 * i);
         if (!mbar_wait(A_EMPTY(as), aph ^ 1u, abort_flag, args.status)) { ok = false; break; }
-        const uint32_t arow = CF::kAOff + as * kABytes + r * 128;
-        const uint32_t sw = static_cast<uint32_t>(r & 7);
-        const uint32_t c0 = static_cast<uint32_t>(4 * half);  // first 16-byte chunk of the half row
-        if (MODE == MOEQ_INT8_ROW) {
-          // 32 int8 codes -> 32 fp16 values (exact)
+        tc_fence_after();
+        const uint32_t tcol = trow + as * kAStageCols;
 #pragma unroll
-          for (int q2 = 0; q2 < 2; ++q2) {
-            const uint4 cw = q2 ? cw1 : cw0;
-            const uint32_t wv[4] = {cw.x, cw.y, cw.z, cw.w};
-            uint32_t o[8];
+        for (int hf = 0; hf < 2; ++hf) {  // two halves of the row: 32 fp16 = 16 columns each
+          uint32_t o[16];
+          if (MODE == MOEQ_INT8_ROW) {
 #pragma unroll
-            for (int wi = 0; wi < 4; ++wi) {
-              const uint32_t bw = wv[wi] ^ 0x80808080u;  // byte = q + 128
-              float f[4];
+            for (int q2 = 0; q2 < 2; ++q2) {
+              const uint4 c4 = cw[2 * hf + q2];
+              const uint32_t wv[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
-              for (int k = 0; k < 4; ++k)
-                f[k] = __fsub_rn(__uint_as_float(__byte_perm(bw, 0x4B000000u, 0x7540u | k)), 8388736.0f);
-              o[2 * wi] = pack_f16(f[0], f[1]);
-              o[2 * wi + 1] = pack_f16(f[2], f[3]);
+              for (int wi = 0; wi < 4; ++wi) {
+                const uint32_t bw = wv[wi] ^ 0x80808080u;  // byte = q + 128
+                float f[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                  f[k] = __fsub_rn(__uint_as_float(__byte_perm(bw, 0x4B000000u, 0x7540u | k)), 8388736.0f);
+                o[8 * q2 + 2 * wi] = pack_f16(f[0], f[1]);
+                o[8 * q2 + 2 * wi + 1] = pack_f16(f[2], f[3]);
+              }
             }
-            const uint32_t cq = c0 + 2 * q2;
-            sts_u4(smem, arow + ((cq ^ sw) << 4), o[0], o[1], o[2], o[3]);
-            sts_u4(smem, arow + (((cq + 1) ^ sw) << 4), o[4], o[5], o[6], o[7]);
-          }
-        } else {
-          const uint32_t wv[4] = {cw0.x, cw0.y, cw0.z, cw0.w};
+          } else {
+            const uint4 c4 = cw[hf];
+            const uint32_t wv[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t hi = (wv[j] >> 4) & 0x0F0F0F0Fu;  // even elements
-            const uint32_t lo = wv[j] & 0x0F0F0F0Fu;         // odd elements
-            uint32_t o[4];
+            for (int j = 0; j < 4; ++j) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint32_t sel = 0x5504u | (static_cast<uint32_t>(k) << 4);
-              float2 c;
-              c.x = __uint_as_float(lds_u32(smem, CF::kLutOff + __byte_perm(hi, lane4, sel)));
-              c.y = __uint_as_float(lds_u32(smem, CF::kLutOff + __byte_perm(lo, lane4, sel)));
-              const float2 w = fmul2(c, a);
-              o[k] = pack_f16(w.x, w.y);
+              for (int k = 0; k < 4; ++k) {
+                // byte k of the word holds elements 2k (high nibble) and 2k+1
+                const uint32_t addr = __byte_perm(wv[j], lane8, 0x5504u | (static_cast<uint32_t>(k) << 4));
+                const float2 c = *reinterpret_cast<const float2 *>(smem + CF::kLutOff + addr);
+                const float2 w = fmul2(c, a);
+                o[4 * j + k] = pack_f16(w.x, w.y);
+              }
             }
-            sts_u4(smem, arow + (((c0 + j) ^ sw) << 4), o[0], o[1], o[2], o[3]);
           }
+          tmem_st_32x32b_x16(tcol + 16u * hf, o);
         }
-        // the proxy fence orders this thread's generic shared-memory accesses (the A
-        // stores, the code loads) before the tensor core's reads and the next TMA write
+        tmem_st_wait();
+        tc_fence_before();
+        // the proxy fence orders this thread's code loads (generic proxy) before the next
+        // TMA write into the slot
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -445,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t b = acc_it & 1u, aph = (acc_it >> 1) & 1u;
       if (!mbar_wait(ACC_FULL(b), aph, abort_flag, args.status)) break;
       tc_fence_after();
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + b * 256u;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + b * kAccCols;
       const int ncols = min(BN / 2, t.count - col0);   // may be <= 0: nothing to do
       const int nch = ncols > 0 ? (ncols + 31) >> 5 : 0;
       if (KIND == 0) {
@@ -577,7 +580,7 @@ cudaError_t launch_moe_gemm(const GemmLaunch &g, int sm_count, cudaStream_t s, i
   const uint32_t code_row = (g.mode == MOEQ_INT8_ROW) ? 64u : 32u;
   for (int i = 0; i < 5; ++i) {
     if (!encode_2d(&maps.b[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g.act, C, g.S, static_cast<uint64_t>(C) * 2,
-                   64, 16u << i, CU_TENSOR_MAP_SWIZZLE_128B))
+                   64, i < 4 ? (16u << i) : 192u, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
   const uint64_t row_bytes = (g.mode == MOEQ_INT8_ROW) ? C : C / 2;

@@ -21,7 +21,7 @@ cudaError_t launch_dequant(const moeq_packed *p, void *out, bool f32, int sm_cou
 
 // route.cu
 constexpr int kRouteChunk = 512;  // (t,k) pairs per routing chunk (one warp, 16 x 32)
-constexpr int kTileN = 256;       // tokens per GEMM tile (UMMA N upper bound)
+constexpr int kTileN = 192;       // tokens per GEMM tile (UMMA N upper bound)
 cudaError_t launch_route(const void *idx, bool idx64, int S, int E, int nchunks,
                          int32_t *counts_chunk, int32_t *chunk_base, int32_t *counts,
                          int32_t *offsets, int32_t *ntile_prefix, int32_t *perm, int32_t *status,
