@@ -41,7 +41,6 @@ namespace moeq {
 constexpr int BM = 128;
 constexpr int BN = kTileN;  // 192
 constexpr int BK = 64;
-constexpr int kBStages = 6;          // token tiles (TMA), freed by the MMA
 constexpr int kAStages = 4;          // dequantized weight stages in TMEM, freed by the MMA
 constexpr uint32_t kAccCols = BN;    // fp32 columns per accumulator
 constexpr uint32_t kACol0 = 2 * kAccCols;  // first TMEM column of the A ring
@@ -57,23 +56,32 @@ constexpr int kMmaWarp = kBProducerWarp + 1;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr int kGroupM = 16;  // m-tiles walked per token tile before moving on (L2 reuse)
 constexpr uint32_t kBBytes = BN * BK * 2;
+constexpr int kMaxExperts = 1024;  // the largest expert count the entry points accept
 // NF4 pair table: for every code byte (two 4-bit codes) the two fp32 levels, one copy
 // per lane: entry (byte, lane) at byte*256 + lane*8, so the address is one byte permute
 // and each lane's 8-byte load hits its own banks.
 constexpr uint32_t kLutBytes = 256 * 256;
 
+// Ring depths.  The packed codes stream from HBM once per token tile, so their ring is
+// the deep one: each dequant group finds several of its stages already landed.  The
+// token tiles are shared by the CTAs walking the same token tile (L2 hits), so four
+// stages cover their latency.
 template <int MODE>
 struct Cfg {
   static constexpr uint32_t kCodeRow = (MODE == MOEQ_INT8_ROW) ? 64 : 32;  // bytes/row/stage
   static constexpr uint32_t kCodeBytes = BM * kCodeRow;
-  static constexpr int kCStages = (MODE == MOEQ_INT8_ROW) ? 8 : 4;  // packed-code tiles
+  static constexpr int kBStages = (MODE == MOEQ_INT8_ROW) ? 5 : 4;   // token tiles, freed by the MMA
+  static constexpr int kCStages = (MODE == MOEQ_INT8_ROW) ? 12 : 14; // packed-code tiles
   static constexpr uint32_t kBOff = 0;
   static constexpr uint32_t kCOff = kBOff + kBStages * kBBytes;
   static constexpr uint32_t kLutOff = kCOff + kCStages * kCodeBytes;
   static constexpr uint32_t kLut = (MODE == MOEQ_INT8_ROW) ? 0 : kLutBytes;
   static constexpr uint32_t kCtrlOff = kLutOff + kLut;
   static constexpr int kNumBars = 2 * kBStages + 2 * kAStages + 2 * kCStages + 5;
-  static constexpr uint32_t kSmem = kCtrlOff + kNumBars * 8 + 16 + 1024;
+  // per-expert token-tile prefix and row offsets, copied once so that every role decodes
+  // its next tile from shared memory instead of a chain of dependent global loads
+  static constexpr uint32_t kTabOff = kCtrlOff + kNumBars * 8 + 16;
+  static constexpr uint32_t kSmem = kTabOff + 2 * (kMaxExperts + 1) * 4 + 1024;
 };
 
 // The 16 NormalFloat-4 levels (fp32), the table the packed codes index.
@@ -110,25 +118,26 @@ struct Tile {
   int e, m, row0, count, nbox;
 };
 
-__device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a) {
+// ntp / offs: the expert tables in shared memory (E + 1 entries each)
+__device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a, const int *ntp, const int *offs) {
   int lo = 0, hi = a.E;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (a.ntp[mid] * a.MT <= tile) lo = mid;
+    if (ntp[mid] * a.MT <= tile) lo = mid;
     else hi = mid;
   }
   Tile t;
   t.e = lo;
-  const int NT = a.ntp[lo + 1] - a.ntp[lo];
-  const int local = tile - a.ntp[lo] * a.MT;
+  const int NT = ntp[lo + 1] - ntp[lo];
+  const int local = tile - ntp[lo] * a.MT;
   const int gfull = NT * kGroupM;
   const int g = local / gfull;
   const int rem = local - g * gfull;
   const int Gg = min(kGroupM, a.MT - g * kGroupM);
   const int nt = rem / Gg;
   t.m = g * kGroupM + (rem - nt * Gg);
-  const int off = a.offsets[lo];
-  const int n_e = a.offsets[lo + 1] - off;
+  const int off = offs[lo];
+  const int n_e = offs[lo + 1] - off;
   const int n0 = nt * BN;
   t.count = min(BN, n_e - n0);
   t.row0 = off + n0;
@@ -153,21 +162,38 @@ __device__ __forceinline__ float2 fmul2(float2 a, float s) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(x), "l"(y));
   return make_float2(__uint_as_float(static_cast<uint32_t>(r)), __uint_as_float(static_cast<uint32_t>(r >> 32)));
 }
+// packed fp16 a - b (round to nearest; exact for the small integers it is used on)
+__device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t *>(&h);
 }
 
+// Decode step s/127 of the double-quantized absmax, kept for the 256-block group it
+// belongs to (a thread walks one weight row, so the group rarely changes).
+struct DqStep {
+  int group = -1;
+  float step = 0.0f;
+};
+
 // fp32 absmax of weight row `wr` (expert e), NF4 block kb
 template <int MODE>
-__device__ __forceinline__ float load_absmax(const GemmArgs &a, int e, int wr, int kb) {
+__device__ __forceinline__ float load_absmax(const GemmArgs &a, int e, int wr, int kb, DqStep &dq) {
   if (MODE == MOEQ_NF4) {
     return __ldg(a.absmax + (static_cast<size_t>(e) * a.R + wr) * (a.C / 64) + kb);
   } else if (MODE == MOEQ_NF4_DQ) {
     const int b = wr * (a.C / 64) + kb;  // block index inside expert e
     const float q = static_cast<float>(__ldg(a.aq + static_cast<size_t>(e) * a.nb + b));
-    const float s = __ldg(a.ascale + static_cast<size_t>(e) * a.nblk + (b >> 8));
-    return __fadd_rn(__fmul_rn(q, __fdiv_rn(s, 127.0f)), __ldg(a.aoff + e));
+    const int g = e * a.nblk + (b >> 8);
+    if (g != dq.group) {
+      dq.group = g;
+      dq.step = __fdiv_rn(__ldg(a.ascale + g), 127.0f);
+    }
+    return __fadd_rn(__fmul_rn(q, dq.step), __ldg(a.aoff + e));
   }
   return 0.0f;
 }
@@ -177,6 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_moe_gemm(const __grid_constant__ TmapSet maps, const GemmArgs args) {
   using CF = Cfg<MODE>;
   constexpr int kCS = CF::kCStages;
+  constexpr int kBStages = CF::kBStages;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, kept as shared-array arithmetic so accesses stay shared loads
   uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -229,6 +256,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           make_float2(kNF4Levels[byte >> 4], kNF4Levels[byte & 15]);
     }
   }
+  int *s_ntp = reinterpret_cast<int *>(smem + CF::kTabOff);
+  int *s_off = s_ntp + (kMaxExperts + 1);
+  for (int i = threadIdx.x; i <= args.E; i += kThreads) {
+    s_ntp[i] = __ldg(args.ntp + i);
+    s_off[i] = __ldg(args.offsets + i);
+  }
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
@@ -242,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int total_tiles = args.ntp[args.E] * args.MT;
+  const int total_tiles = s_ntp[args.E] * args.MT;
   const int nk = args.nk;
 
   if (warp == kCodeProducerWarp) {
@@ -251,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-        const Tile t = decode_tile(tile, args);
+        const Tile t = decode_tile(tile, args, s_ntp, s_off);
         int y0, y1;
         if (KIND == 0) {
           y0 = t.e * args.R + t.m * 64;
@@ -286,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-        const Tile t = decode_tile(tile, args);
+        const Tile t = decode_tile(tile, args, s_ntp, s_off);
         const uint32_t tx = box_rows(t.nbox) * 128u;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % kBStages, ph = (it / kBStages) & 1u;
@@ -311,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0, acc_it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++acc_it) {
-        const Tile t = decode_tile(tile, args);
+        const Tile t = decode_tile(tile, args, s_ntp, s_off);
         const uint32_t b = acc_it & 1u, aph = (acc_it >> 1) & 1u;
         if (!mbar_wait(ACC_EMPTY(b), aph ^ 1u, abort_flag, args.status)) break;
         tc_fence_after();
@@ -358,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-      const Tile t = decode_tile(tile, args);
+      const Tile t = decode_tile(tile, args, s_ntp, s_off);
       int wr, cr;  // weight row inside the expert, row inside the staged code tile
       if (KIND == 0) {
         const int sgate = r & 1, i = r >> 1;
@@ -370,13 +403,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float a_pref = 0.f;
       bool have_pref = false;
+      DqStep dq;
       for (int kb = 0; kb < nk; ++kb, ++it) {
         if (static_cast<int>(it % kDequantGroups) != group) continue;
         float a = 0.f;
         if (MODE != MOEQ_INT8_ROW) {
-          a = have_pref ? a_pref : load_absmax<MODE>(args, t.e, wr, kb);
+          a = have_pref ? a_pref : load_absmax<MODE>(args, t.e, wr, kb, dq);
           have_pref = kb + kDequantGroups < nk;
-          if (have_pref) a_pref = load_absmax<MODE>(args, t.e, wr, kb + kDequantGroups);
+          if (have_pref) a_pref = load_absmax<MODE>(args, t.e, wr, kb + kDequantGroups, dq);
         }
         const uint32_t cs = it % kCS, cph = (it / kCS) & 1u;
         const uint32_t as = it % kAStages, aph = (it / kAStages) & 1u;
@@ -399,13 +433,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t wv[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
               for (int wi = 0; wi < 4; ++wi) {
-                const uint32_t bw = wv[wi] ^ 0x80808080u;  // byte = q + 128
-                float f[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                  f[k] = __fsub_rn(__uint_as_float(__byte_perm(bw, 0x4B000000u, 0x7540u | k)), 8388736.0f);
-                o[8 * q2 + 2 * wi] = pack_f16(f[0], f[1]);
-                o[8 * q2 + 2 * wi + 1] = pack_f16(f[2], f[3]);
+                // fp16 0x64XX is 1024 + XX (ulp 1 on [1024, 2048)), so with byte = q + 128
+                // the pair (0x64 byte0, 0x64 byte1) minus 1152 is (q0, q1), exactly
+                const uint32_t bw = wv[wi] ^ 0x80808080u;
+                o[8 * q2 + 2 * wi] = hsub2_u32(__byte_perm(bw, 0x64646464u, 0x4140u), 0x64806480u);
+                o[8 * q2 + 2 * wi + 1] = hsub2_u32(__byte_perm(bw, 0x64646464u, 0x4342u), 0x64806480u);
               }
             }
           } else {
@@ -444,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = quad * 32 + lane;
     uint32_t acc_it = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++acc_it) {
-      const Tile t = decode_tile(tile, args);
+      const Tile t = decode_tile(tile, args, s_ntp, s_off);
       const uint32_t b = acc_it & 1u, aph = (acc_it >> 1) & 1u;
       if (!mbar_wait(ACC_FULL(b), aph, abort_flag, args.status)) break;
       tc_fence_after();
