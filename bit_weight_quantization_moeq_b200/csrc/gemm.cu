@@ -41,14 +41,23 @@ namespace moeq {
 constexpr int BM = 128;
 constexpr int BN = kTileN;  // 192
 constexpr int BK = 64;
-constexpr int kAStages = 4;          // dequantized weight stages in TMEM, freed by the MMA
+// The operand rings advance in pairs of K stages: one pair = 2 x 64 of K = 8 MMAs of
+// K = 16, and one full/empty barrier pair covers both the A and B halves of a pair.  The
+// single MMA-issuing thread then waits and commits once per 8 MMAs: at N = 192 an MMA
+// runs ~96 cycles and the tensor core queues few instructions, so a wait and a commit
+// per 4 MMAs leave the tensor pipe idle between stages.
+constexpr int kPairSlots = 2;        // pairs in flight
+constexpr int kAStages = 2 * kPairSlots;  // dequantized weight stages in TMEM
+constexpr int kBStages = 2 * kPairSlots;  // token tiles in shared memory
 constexpr uint32_t kAccCols = BN;    // fp32 columns per accumulator
 constexpr uint32_t kACol0 = 2 * kAccCols;  // first TMEM column of the A ring
 constexpr uint32_t kAStageCols = 32;       // 64 fp16 per row = 32 columns
+static_assert(kACol0 + kAStages * kAStageCols <= 512, "accumulators and A ring fit in TMEM");
 constexpr int kEpiWarps = 8;
 constexpr int kDequantGroups = 4;    // groups take K stages in turn
 constexpr int kGroupWarps = 4;       // per group: 128 rows, one per thread
 constexpr int kDequantWarps = kDequantGroups * kGroupWarps;
+static_assert((kDequantGroups & (kDequantGroups - 1)) == 0, "groups are picked with a mask");
 constexpr int kDequantThread0 = kEpiWarps * 32;
 constexpr int kCodeProducerWarp = kEpiWarps + kDequantWarps;
 constexpr int kBProducerWarp = kCodeProducerWarp + 1;
@@ -64,24 +73,24 @@ constexpr uint32_t kLutBytes = 256 * 256;
 
 // Ring depths.  The packed codes stream from HBM once per token tile, so their ring is
 // the deep one: each dequant group finds several of its stages already landed.  The
-// token tiles are shared by the CTAs walking the same token tile (L2 hits), so four
-// stages cover their latency.
+// token tiles are shared by the CTAs walking the same token tile (L2 hits), so two pairs
+// of stages cover their latency.
 template <int MODE>
 struct Cfg {
   static constexpr uint32_t kCodeRow = (MODE == MOEQ_INT8_ROW) ? 64 : 32;  // bytes/row/stage
   static constexpr uint32_t kCodeBytes = BM * kCodeRow;
-  static constexpr int kBStages = (MODE == MOEQ_INT8_ROW) ? 5 : 4;   // token tiles, freed by the MMA
-  static constexpr int kCStages = (MODE == MOEQ_INT8_ROW) ? 12 : 14; // packed-code tiles
+  static constexpr int kCStages = (MODE == MOEQ_INT8_ROW) ? 14 : 14; // packed-code tiles
   static constexpr uint32_t kBOff = 0;
   static constexpr uint32_t kCOff = kBOff + kBStages * kBBytes;
   static constexpr uint32_t kLutOff = kCOff + kCStages * kCodeBytes;
   static constexpr uint32_t kLut = (MODE == MOEQ_INT8_ROW) ? 0 : kLutBytes;
   static constexpr uint32_t kCtrlOff = kLutOff + kLut;
-  static constexpr int kNumBars = 2 * kBStages + 2 * kAStages + 2 * kCStages + 5;
+  static constexpr int kNumBars = 2 * kPairSlots + 2 * kCStages + 5;
   // per-expert token-tile prefix and row offsets, copied once so that every role decodes
   // its next tile from shared memory instead of a chain of dependent global loads
   static constexpr uint32_t kTabOff = kCtrlOff + kNumBars * 8 + 16;
   static constexpr uint32_t kSmem = kTabOff + 2 * (kMaxExperts + 1) * 4 + 1024;
+  static_assert(kSmem <= 232448, "shared memory per block");
 };
 
 // The 16 NormalFloat-4 levels (fp32), the table the packed codes index.
@@ -203,22 +212,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_moe_gemm(const __grid_constant__ TmapSet maps, const GemmArgs args) {
   using CF = Cfg<MODE>;
   constexpr int kCS = CF::kCStages;
-  constexpr int kBStages = CF::kBStages;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, kept as shared-array arithmetic so accesses stay shared loads
   uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
   uint8_t *ctrl = smem + CF::kCtrlOff;
   const uint32_t bar0 = smem_u32(ctrl);
-  // barriers: token ring full/empty, A ring full/empty, code ring full/empty,
-  // accumulator full/empty (x2), drain
-  auto B_FULL = [&](int i) -> uint32_t { return bar0 + 8u * i; };
-  auto B_EMPTY = [&](int i) -> uint32_t { return bar0 + 8u * (kBStages + i); };
-  auto A_FULL = [&](int i) -> uint32_t { return bar0 + 8u * (2 * kBStages + i); };
-  auto A_EMPTY = [&](int i) -> uint32_t { return bar0 + 8u * (2 * kBStages + kAStages + i); };
-  auto C_FULL = [&](int i) -> uint32_t { return bar0 + 8u * (2 * kBStages + 2 * kAStages + i); };
-  auto C_EMPTY = [&](int i) -> uint32_t { return bar0 + 8u * (2 * kBStages + 2 * kAStages + kCS + i); };
-  constexpr int kAcc0 = 2 * kBStages + 2 * kAStages + 2 * kCS;
+  // barriers: operand pair slots full/empty (both K stages of a pair, A in TMEM and B in
+  // shared memory), code ring full/empty, accumulator full/empty (x2), drain
+  auto FULL = [&](uint32_t i) -> uint32_t { return bar0 + 8u * i; };
+  auto EMPTY = [&](uint32_t i) -> uint32_t { return bar0 + 8u * (kPairSlots + i); };
+  auto C_FULL = [&](uint32_t i) -> uint32_t { return bar0 + 8u * (2 * kPairSlots + i); };
+  auto C_EMPTY = [&](uint32_t i) -> uint32_t { return bar0 + 8u * (2 * kPairSlots + kCS + i); };
+  constexpr int kAcc0 = 2 * kPairSlots + 2 * kCS;
   auto ACC_FULL = [&](int b) -> uint32_t { return bar0 + 8u * (kAcc0 + b); };
   auto ACC_EMPTY = [&](int b) -> uint32_t { return bar0 + 8u * (kAcc0 + 2 + b); };
   const uint32_t DRAIN = bar0 + 8u * (kAcc0 + 4);
@@ -228,13 +234,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kBStages; ++i) {
-      mbar_init(B_FULL(i), 1);        // producer arrive + tx bytes
-      mbar_init(B_EMPTY(i), 1);       // MMA commit
-    }
-    for (int i = 0; i < kAStages; ++i) {
-      mbar_init(A_FULL(i), kGroupWarps);  // one arrival per warp of the dequant group
-      mbar_init(A_EMPTY(i), 1);           // MMA commit
+    for (int i = 0; i < kPairSlots; ++i) {
+      // token producer (arrive + tx bytes) and, per K stage of the pair, one arrival per
+      // warp of the dequant group that wrote it (a lone last stage arrives twice)
+      mbar_init(FULL(i), 2 * kGroupWarps + 1);
+      mbar_init(EMPTY(i), 1);             // MMA commit
     }
     for (int i = 0; i < kCS; ++i) {
       mbar_init(C_FULL(i), 1);            // producer arrive + tx bytes
@@ -314,25 +318,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp == kBProducerWarp) {
-    // ---------------- token-tile producer ----------------
+    // ---------------- token-tile producer (one pair of K stages at a time) ----------------
     if (lane == 0) {
-      uint32_t it = 0;
+      uint32_t pr = 0;  // pairs issued by this CTA
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
         const Tile t = decode_tile(tile, args, s_ntp, s_off);
-        const uint32_t tx = box_rows(t.nbox) * 128u;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
-          const uint32_t s = it % kBStages, ph = (it / kBStages) & 1u;
-          if (!mbar_wait(B_EMPTY(s), ph ^ 1u, abort_flag, args.status)) { ok = false; break; }
-          mbar_arrive_expect_tx(B_FULL(s), tx);
-          tma_load_2d(sbase + CF::kBOff + s * kBBytes, &maps.b[t.nbox], kb * BK, t.row0, B_FULL(s));
+        const uint32_t box = box_rows(t.nbox) * 128u;
+        for (int kb = 0; kb < nk; kb += 2, ++pr) {
+          const uint32_t ps = pr & 1u, ph = (pr >> 1) & 1u;
+          if (!mbar_wait(EMPTY(ps), ph ^ 1u, abort_flag, args.status)) { ok = false; break; }
+          const int nst = min(2, nk - kb);
+          mbar_arrive_expect_tx(FULL(ps), box * nst);
+          for (int h = 0; h < nst; ++h)
+            tma_load_2d(sbase + CF::kBOff + (2 * ps + h) * kBBytes, &maps.b[t.nbox], (kb + h) * BK, t.row0,
+                        FULL(ps));
         }
       }
-      const uint32_t n = it < static_cast<uint32_t>(kBStages) ? it : static_cast<uint32_t>(kBStages);
+      // drain: the copies of the last pairs land before the CTA may exit (on the normal
+      // path the MMA has consumed every pair already)
+      const uint32_t n = pr < static_cast<uint32_t>(kPairSlots) ? pr : static_cast<uint32_t>(kPairSlots);
       for (uint32_t d = 0; d < n; ++d) {
-        const uint32_t j = it - 1 - d;
+        const uint32_t j = pr - 1 - d;
         const uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(B_FULL(j % kBStages), (j / kBStages) & 1u)) {
+        while (!mbar_try_wait(FULL(j & 1u), (j >> 1) & 1u)) {
           if (globaltimer() - t0 > kWaitLimitNs) break;
         }
       }
@@ -341,8 +350,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      uint32_t it = 0, acc_it = 0;
+      uint32_t pr = 0, acc_it = 0;
       bool ok = true;
+      bool ready = false;  // the next pair's barrier was already seen complete
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++acc_it) {
         const Tile t = decode_tile(tile, args, s_ntp, s_off);
         const uint32_t b = acc_it & 1u, aph = (acc_it >> 1) & 1u;
@@ -351,24 +361,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d_tmem = tmem_base + b * kAccCols;
         const uint32_t n_mma = static_cast<uint32_t>((t.count + 15) & ~15);
         const uint32_t idesc = umma_idesc_f16_m128(n_mma);
-        for (int kb = 0; kb < nk; ++kb, ++it) {
-          const uint32_t bs = it % kBStages, bph = (it / kBStages) & 1u;
-          const uint32_t as = it % kAStages, aph2 = (it / kAStages) & 1u;
-          if (!mbar_wait(B_FULL(bs), bph, abort_flag, args.status) ||
-              !mbar_wait(A_FULL(as), aph2, abort_flag, args.status)) {
-            ok = false;
-            break;
-          }
+        for (int kb = 0; kb < nk; kb += 2, ++pr) {
+          const uint32_t ps = pr & 1u, ph = (pr >> 1) & 1u;
+          if (!ready && !mbar_wait(FULL(ps), ph, abort_flag, args.status)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_tmem = tmem_base + kACol0 + as * kAStageCols;
-          const uint64_t bdesc = umma_desc_sw128(sbase + CF::kBOff + bs * kBBytes);
+          // look at the next pair's barrier now, while this pair's MMAs queue up
+          ready = mbar_try_wait(FULL(ps ^ 1u), ((pr + 1) >> 1) & 1u);
+          const int nst = min(2, nk - kb);
+          for (int h = 0; h < nst; ++h) {
+            const uint32_t a_tmem = tmem_base + kACol0 + (2 * ps + h) * kAStageCols;
+            const uint64_t bdesc = umma_desc_sw128(sbase + CF::kBOff + (2 * ps + h) * kBBytes);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            // K = 16 per MMA: +8 TMEM columns of A, +32 bytes (+2 in the start field) of B
-            umma_f16_ts(d_tmem, a_tmem + 8u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
+            for (int k = 0; k < BK / 16; ++k) {
+              // K = 16 per MMA: +8 TMEM columns of A, +32 bytes (+2 in the start field) of B
+              umma_f16_ts(d_tmem, a_tmem + 8u * k, bdesc + 2u * k, idesc, (kb | h | k) != 0 ? 1u : 0u);
+            }
           }
-          umma_commit(B_EMPTY(bs));
-          umma_commit(A_EMPTY(as));
+          umma_commit(EMPTY(ps));
         }
         if (!ok) break;
         umma_commit(ACC_FULL(b));
@@ -383,14 +392,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= kEpiWarps) {
     // ---------------- dequant (four groups, K stages in turn) ----------------
+    // A group decodes its stage into registers first and only then waits for the TMEM
+    // slot, so that the slot (freed when the MMAs of the pair two back complete) is
+    // refilled with a few tcgen05.st.
     const int dt = threadIdx.x - kDequantThread0;
     const int group = dt / (kGroupWarps * 32);
     const int r = dt - group * (kGroupWarps * 32);  // tile row = TMEM lane (warp%4 quadrant)
     const uint32_t lane8 = static_cast<uint32_t>(lane) * 8u;
     const uint32_t trow = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kACol0;
-    uint32_t it = 0;
+    uint32_t it = 0, cs = 0, cph = 0, pr0 = 0;  // K stages, code slot/phase, pairs before this tile
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, pr0 += (nk + 1) >> 1) {
       const Tile t = decode_tile(tile, args, s_ntp, s_off);
       int wr, cr;  // weight row inside the expert, row inside the staged code tile
       if (KIND == 0) {
@@ -405,44 +417,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool have_pref = false;
       DqStep dq;
       for (int kb = 0; kb < nk; ++kb, ++it) {
-        if (static_cast<int>(it % kDequantGroups) != group) continue;
+        const uint32_t my_cs = cs, my_cph = cph;
+        if (++cs == static_cast<uint32_t>(kCS)) { cs = 0; cph ^= 1u; }
+        if (static_cast<int>(it & (kDequantGroups - 1)) != group) continue;
         float a = 0.f;
         if (MODE != MOEQ_INT8_ROW) {
           a = have_pref ? a_pref : load_absmax<MODE>(args, t.e, wr, kb, dq);
           have_pref = kb + kDequantGroups < nk;
           if (have_pref) a_pref = load_absmax<MODE>(args, t.e, wr, kb + kDequantGroups, dq);
         }
-        const uint32_t cs = it % kCS, cph = (it / kCS) & 1u;
-        const uint32_t as = it % kAStages, aph = (it / kAStages) & 1u;
-        if (!mbar_wait(C_FULL(cs), cph, abort_flag, args.status)) { ok = false; break; }
+        if (!mbar_wait(C_FULL(my_cs), my_cph, abort_flag, args.status)) { ok = false; break; }
         // this thread's codes: its row of the stage, 32 bytes (NF4) or 64 bytes (int8)
-        const uint32_t crow = CF::kCOff + cs * CF::kCodeBytes + cr * CF::kCodeRow;
+        const uint32_t crow = CF::kCOff + my_cs * CF::kCodeBytes + cr * CF::kCodeRow;
         uint4 cw[CF::kCodeRow / 16];
 #pragma unroll
         for (int i = 0; i < static_cast<int>(CF::kCodeRow / 16); ++i) cw[i] = lds_u4(smem, crow + 16 * i);
-        if (!mbar_wait(A_EMPTY(as), aph ^ 1u, abort_flag, args.status)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t tcol = trow + as * kAStageCols;
+        // the codes are in registers: hand the slot back to the producer (the proxy fence
+        // orders these generic-proxy reads before its next TMA write into the slot)
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(C_EMPTY(my_cs));
+        uint32_t o[32];  // the row's 64 fp16 weights, two per word, in K order
+        if (MODE == MOEQ_INT8_ROW) {
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {  // two halves of the row: 32 fp16 = 16 columns each
-          uint32_t o[16];
-          if (MODE == MOEQ_INT8_ROW) {
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t wv[4] = {cw[q].x, cw[q].y, cw[q].z, cw[q].w};
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-              const uint4 c4 = cw[2 * hf + q2];
-              const uint32_t wv[4] = {c4.x, c4.y, c4.z, c4.w};
-#pragma unroll
-              for (int wi = 0; wi < 4; ++wi) {
-                // fp16 0x64XX is 1024 + XX (ulp 1 on [1024, 2048)), so with byte = q + 128
-                // the pair (0x64 byte0, 0x64 byte1) minus 1152 is (q0, q1), exactly
-                const uint32_t bw = wv[wi] ^ 0x80808080u;
-                o[8 * q2 + 2 * wi] = hsub2_u32(__byte_perm(bw, 0x64646464u, 0x4140u), 0x64806480u);
-                o[8 * q2 + 2 * wi + 1] = hsub2_u32(__byte_perm(bw, 0x64646464u, 0x4342u), 0x64806480u);
-              }
+            for (int wi = 0; wi < 4; ++wi) {
+              // fp16 0x64XX is 1024 + XX (ulp 1 on [1024, 2048)), so with byte = q + 128
+              // the pair (0x64 byte0, 0x64 byte1) minus 1152 is (q0, q1), exactly
+              const uint32_t bw = wv[wi] ^ 0x80808080u;
+              o[8 * q + 2 * wi] = hsub2_u32(__byte_perm(bw, 0x64646464u, 0x4140u), 0x64806480u);
+              o[8 * q + 2 * wi + 1] = hsub2_u32(__byte_perm(bw, 0x64646464u, 0x4342u), 0x64806480u);
             }
-          } else {
-            const uint4 c4 = cw[hf];
-            const uint32_t wv[4] = {c4.x, c4.y, c4.z, c4.w};
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const uint32_t wv[4] = {cw[q].x, cw[q].y, cw[q].z, cw[q].w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
 #pragma unroll
@@ -451,21 +463,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t addr = __byte_perm(wv[j], lane8, 0x5504u | (static_cast<uint32_t>(k) << 4));
                 const float2 c = *reinterpret_cast<const float2 *>(smem + CF::kLutOff + addr);
                 const float2 w = fmul2(c, a);
-                o[4 * j + k] = pack_f16(w.x, w.y);
+                o[16 * q + 4 * j + k] = pack_f16(w.x, w.y);
               }
             }
           }
-          tmem_st_32x32b_x16(tcol + 16u * hf, o);
         }
+        // this stage's A slot: half (kb & 1) of the pair's slot
+        const uint32_t pr = pr0 + (kb >> 1), ps = pr & 1u, ph = (pr >> 1) & 1u;
+        if (!mbar_wait(EMPTY(ps), ph ^ 1u, abort_flag, args.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tcol = trow + (2 * ps + (kb & 1)) * kAStageCols;
+        tmem_st_32x32b_x16(tcol, *reinterpret_cast<const uint32_t(*)[16]>(o));
+        tmem_st_32x32b_x16(tcol + 16u, *reinterpret_cast<const uint32_t(*)[16]>(o + 16));
         tmem_st_wait();
         tc_fence_before();
-        // the proxy fence orders this thread's code loads (generic proxy) before the next
-        // TMA write into the slot
-        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(A_FULL(as));
-          mbar_arrive(C_EMPTY(cs));
+          // a lone last stage (odd K / 64) stands for both halves of its pair
+          if ((nk & 1) && kb == nk - 1) mbar_arrive_cnt(FULL(ps), 2);
+          else mbar_arrive(FULL(ps));
         }
       }
     }

@@ -86,9 +86,10 @@ def test_route_drops_bad_indices_and_reports():
 @pytest.mark.parametrize("mode", [0, 1, 2])
 @pytest.mark.parametrize("E,H,I,T,K", [
     (8, 256, 128, 64, 2),       # the tiny workload's shapes
-    (6, 384, 192, 700, 2),      # several m-tiles, one ragged token tile per expert
-    (4, 256, 128, 1500, 2),     # several token tiles per expert (256, 256, ragged)
+    (6, 384, 192, 700, 2),      # several m-tiles; odd K / 64 in down (a lone last K stage)
+    (4, 256, 128, 1500, 2),     # several token tiles per expert (full 192-wide ones, ragged)
     (16, 512, 256, 37, 8),      # few tokens per expert (small UMMA N)
+    (4, 128, 64, 300, 2),       # the smallest shapes: one K stage in down, one m-tile
 ])
 def test_forward_parity(mode, E, H, I, T, K):
     inp = make_inputs(E, H, I, T, K, seed=100 * E + T + mode, outliers=(mode == 2))
