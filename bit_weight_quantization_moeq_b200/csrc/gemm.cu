@@ -46,9 +46,12 @@ constexpr int BK = 64;
 // single MMA-issuing thread then waits and commits once per 8 MMAs: at N = 192 an MMA
 // runs ~96 cycles and the tensor core queues few instructions, so a wait and a commit
 // per 4 MMAs leave the tensor pipe idle between stages.
-constexpr int kPairSlots = 2;        // pairs in flight
+constexpr int kPairSlots = 2;        // pairs of A stages in TMEM
 constexpr int kAStages = 2 * kPairSlots;  // dequantized weight stages in TMEM
-constexpr int kBStages = 2 * kPairSlots;  // token tiles in shared memory
+constexpr int kBPairs = 3;           // pairs of token tiles in shared memory (a 48 KB pair
+                                     // takes ~1000 cycles to land: two pairs of lead)
+constexpr int kBStages = 2 * kBPairs;
+constexpr int kDonePairs = 6;        // pair-completion barriers (a multiple of 2 and 3)
 constexpr uint32_t kAccCols = BN;    // fp32 columns per accumulator
 constexpr uint32_t kACol0 = 2 * kAccCols;  // first TMEM column of the A ring
 constexpr uint32_t kAStageCols = 32;       // 64 fp16 per row = 32 columns
@@ -62,30 +65,30 @@ constexpr int kDequantThread0 = kEpiWarps * 32;
 constexpr int kCodeProducerWarp = kEpiWarps + kDequantWarps;
 constexpr int kBProducerWarp = kCodeProducerWarp + 1;
 constexpr int kMmaWarp = kBProducerWarp + 1;
-constexpr int kThreads = (kMmaWarp + 1) * 32;
+constexpr int kRelayWarp = kMmaWarp + 1;
+constexpr int kThreads = (kRelayWarp + 1) * 32;
 constexpr int kGroupM = 16;  // m-tiles walked per token tile before moving on (L2 reuse)
 constexpr uint32_t kBBytes = BN * BK * 2;
 constexpr int kMaxExperts = 1024;  // the largest expert count the entry points accept
-// NF4 pair table: for every code byte (two 4-bit codes) the two fp32 levels, one copy
-// per lane: entry (byte, lane) at byte*256 + lane*8, so the address is one byte permute
-// and each lane's 8-byte load hits its own banks.
-constexpr uint32_t kLutBytes = 256 * 256;
+// NF4 pair table: for every code byte (two 4-bit codes) the two levels as an fp16 pair,
+// one copy per lane: entry (byte, lane) at byte*128 + lane*4, so a warp's 32 lookups hit
+// 32 different banks, and the address is a byte permute and a shift.
+constexpr uint32_t kLutBytes = 256 * 128;
 
 // Ring depths.  The packed codes stream from HBM once per token tile, so their ring is
-// the deep one: each dequant group finds several of its stages already landed.  The
-// token tiles are shared by the CTAs walking the same token tile (L2 hits), so two pairs
-// of stages cover their latency.
+// the deep one: each dequant group finds several of its stages already landed (a group
+// copies its codes to registers and frees the slot at once).
 template <int MODE>
 struct Cfg {
   static constexpr uint32_t kCodeRow = (MODE == MOEQ_INT8_ROW) ? 64 : 32;  // bytes/row/stage
   static constexpr uint32_t kCodeBytes = BM * kCodeRow;
-  static constexpr int kCStages = (MODE == MOEQ_INT8_ROW) ? 14 : 14; // packed-code tiles
+  static constexpr int kCStages = (MODE == MOEQ_INT8_ROW) ? 8 : 10;  // packed-code tiles
   static constexpr uint32_t kBOff = 0;
   static constexpr uint32_t kCOff = kBOff + kBStages * kBBytes;
   static constexpr uint32_t kLutOff = kCOff + kCStages * kCodeBytes;
   static constexpr uint32_t kLut = (MODE == MOEQ_INT8_ROW) ? 0 : kLutBytes;
   static constexpr uint32_t kCtrlOff = kLutOff + kLut;
-  static constexpr int kNumBars = 2 * kPairSlots + 2 * kCStages + 5;
+  static constexpr int kNumBars = kPairSlots + kDonePairs + kBPairs + 2 * kCStages + 5;
   // per-expert token-tile prefix and row offsets, copied once so that every role decodes
   // its next tile from shared memory instead of a chain of dependent global loads
   static constexpr uint32_t kTabOff = kCtrlOff + kNumBars * 8 + 16;
@@ -163,23 +166,11 @@ __device__ __forceinline__ uint4 lds_u4(const uint8_t *smem, uint32_t off) {
   return *reinterpret_cast<const uint4 *>(smem + off);
 }
 
-// (a.x * s, a.y * s) with one packed fp32x2 multiply, each product rounded once
-__device__ __forceinline__ float2 fmul2(float2 a, float s) {
-  uint64_t r;
-  const uint64_t x = (static_cast<uint64_t>(__float_as_uint(a.y)) << 32) | __float_as_uint(a.x);
-  const uint64_t y = (static_cast<uint64_t>(__float_as_uint(s)) << 32) | __float_as_uint(s);
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(x), "l"(y));
-  return make_float2(__uint_as_float(static_cast<uint32_t>(r)), __uint_as_float(static_cast<uint32_t>(r >> 32)));
-}
 // packed fp16 a - b (round to nearest; exact for the small integers it is used on)
 __device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
   uint32_t r;
   asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
-}
-__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
-  const __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t *>(&h);
 }
 
 // Decode step s/127 of the double-quantized absmax, kept for the 256-block group it
@@ -218,13 +209,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   uint8_t *ctrl = smem + CF::kCtrlOff;
   const uint32_t bar0 = smem_u32(ctrl);
-  // barriers: operand pair slots full/empty (both K stages of a pair, A in TMEM and B in
-  // shared memory), code ring full/empty, accumulator full/empty (x2), drain
+  // barriers: FULL (a pair's A stages are in TMEM and its token tiles have landed: what
+  // the MMA waits on), DONE (the MMAs of pair j have completed, on DONE(j % 6)), BFULL
+  // (a pair's token-tile copies), code ring full/empty, accumulator full/empty (x2), drain
   auto FULL = [&](uint32_t i) -> uint32_t { return bar0 + 8u * i; };
-  auto EMPTY = [&](uint32_t i) -> uint32_t { return bar0 + 8u * (kPairSlots + i); };
-  auto C_FULL = [&](uint32_t i) -> uint32_t { return bar0 + 8u * (2 * kPairSlots + i); };
-  auto C_EMPTY = [&](uint32_t i) -> uint32_t { return bar0 + 8u * (2 * kPairSlots + kCS + i); };
-  constexpr int kAcc0 = 2 * kPairSlots + 2 * kCS;
+  auto DONE = [&](uint32_t i) -> uint32_t { return bar0 + 8u * (kPairSlots + i); };
+  auto BFULL = [&](uint32_t i) -> uint32_t { return bar0 + 8u * (kPairSlots + kDonePairs + i); };
+  constexpr int kC0 = kPairSlots + kDonePairs + kBPairs;
+  auto C_FULL = [&](uint32_t i) -> uint32_t { return bar0 + 8u * (kC0 + i); };
+  auto C_EMPTY = [&](uint32_t i) -> uint32_t { return bar0 + 8u * (kC0 + kCS + i); };
+  constexpr int kAcc0 = kC0 + 2 * kCS;
   auto ACC_FULL = [&](int b) -> uint32_t { return bar0 + 8u * (kAcc0 + b); };
   auto ACC_EMPTY = [&](int b) -> uint32_t { return bar0 + 8u * (kAcc0 + 2 + b); };
   const uint32_t DRAIN = bar0 + 8u * (kAcc0 + 4);
@@ -235,11 +229,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kPairSlots; ++i) {
-      // token producer (arrive + tx bytes) and, per K stage of the pair, one arrival per
-      // warp of the dequant group that wrote it (a lone last stage arrives twice)
+      // the relay (token tiles landed) and, per K stage of the pair, one arrival per warp
+      // of the dequant group that wrote it (a lone last stage arrives twice)
       mbar_init(FULL(i), 2 * kGroupWarps + 1);
-      mbar_init(EMPTY(i), 1);             // MMA commit
     }
+    for (int i = 0; i < kDonePairs; ++i) mbar_init(DONE(i), 1);  // MMA commit
+    for (int i = 0; i < kBPairs; ++i) mbar_init(BFULL(i), 1);    // producer arrive + tx bytes
     for (int i = 0; i < kCS; ++i) {
       mbar_init(C_FULL(i), 1);            // producer arrive + tx bytes
       mbar_init(C_EMPTY(i), kGroupWarps); // the group has read the codes
@@ -256,8 +251,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // NF4 pair table (see kLutBytes): entry (byte, lane) = (c[byte >> 4], c[byte & 15])
     for (int i = threadIdx.x; i < 256 * 32; i += kThreads) {
       const int byte = i >> 5, l = i & 31;
-      *reinterpret_cast<float2 *>(smem + CF::kLutOff + byte * 256 + l * 8) =
-          make_float2(kNF4Levels[byte >> 4], kNF4Levels[byte & 15]);
+      *reinterpret_cast<__half2 *>(smem + CF::kLutOff + byte * 128 + l * 4) =
+          __floats2half2_rn(kNF4Levels[byte >> 4], kNF4Levels[byte & 15]);
     }
   }
   int *s_ntp = reinterpret_cast<int *>(smem + CF::kTabOff);
@@ -326,23 +321,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile t = decode_tile(tile, args, s_ntp, s_off);
         const uint32_t box = box_rows(t.nbox) * 128u;
         for (int kb = 0; kb < nk; kb += 2, ++pr) {
-          const uint32_t ps = pr & 1u, ph = (pr >> 1) & 1u;
-          if (!mbar_wait(EMPTY(ps), ph ^ 1u, abort_flag, args.status)) { ok = false; break; }
+          // the slot pair pr % 3 was last read by the MMAs of pair pr - 3
+          if (pr >= static_cast<uint32_t>(kBPairs)) {
+            const uint32_t j = pr - kBPairs;
+            if (!mbar_wait(DONE(j % kDonePairs), (j / kDonePairs) & 1u, abort_flag, args.status)) { ok = false; break; }
+          }
+          const uint32_t bs = pr % kBPairs;
           const int nst = min(2, nk - kb);
-          mbar_arrive_expect_tx(FULL(ps), box * nst);
+          mbar_arrive_expect_tx(BFULL(bs), box * nst);
           for (int h = 0; h < nst; ++h)
-            tma_load_2d(sbase + CF::kBOff + (2 * ps + h) * kBBytes, &maps.b[t.nbox], (kb + h) * BK, t.row0,
-                        FULL(ps));
+            tma_load_2d(sbase + CF::kBOff + (2 * bs + h) * kBBytes, &maps.b[t.nbox], (kb + h) * BK, t.row0,
+                        BFULL(bs));
         }
       }
-      // drain: the copies of the last pairs land before the CTA may exit (on the normal
-      // path the MMA has consumed every pair already)
-      const uint32_t n = pr < static_cast<uint32_t>(kPairSlots) ? pr : static_cast<uint32_t>(kPairSlots);
+      // drain: the copies of the last pairs land before the CTA may exit
+      const uint32_t n = pr < static_cast<uint32_t>(kBPairs) ? pr : static_cast<uint32_t>(kBPairs);
       for (uint32_t d = 0; d < n; ++d) {
         const uint32_t j = pr - 1 - d;
         const uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(FULL(j & 1u), (j >> 1) & 1u)) {
+        while (!mbar_try_wait(BFULL(j % kBPairs), (j / kBPairs) & 1u)) {
           if (globaltimer() - t0 > kWaitLimitNs) break;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == kRelayWarp) {
+    // ---------------- relay: a pair's token tiles have landed -> its FULL barrier ----------------
+    // (the MMA thread then waits on a single barrier per pair; the token ring is deeper
+    // than the A ring, so its copies are tracked on barriers of their own)
+    if (lane == 0) {
+      uint32_t pr = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        for (int kb = 0; kb < nk; kb += 2, ++pr) {
+          if (!mbar_wait(BFULL(pr % kBPairs), (pr / kBPairs) & 1u, abort_flag, args.status)) { ok = false; break; }
+          // this arrival must count toward pair pr: FULL(pr % 2) has to be done with pair pr - 2
+          if (pr >= 2 && !mbar_wait(FULL(pr & 1u), ((pr - 2) >> 1) & 1u, abort_flag, args.status)) { ok = false; break; }
+          mbar_arrive(FULL(pr & 1u));
         }
       }
     }
@@ -350,7 +365,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      uint32_t pr = 0, acc_it = 0;
+      // The issue loop is kept minimal: the tensor core queues few MMAs, so every cycle
+      // this thread spends between two MMAs can leave the tensor pipe idle.  Operand
+      // addresses advance by adding to precomputed bases (the descriptor's start field is
+      // the shared-memory address >> 4; no carry leaves its 14 bits below 256 KB).
+      const uint32_t a_base = tmem_base + kACol0;
+      const uint64_t b_base = umma_desc_sw128(sbase + CF::kBOff);
+      constexpr uint32_t kBStep = kBBytes >> 4;  // one token tile in descriptor units
+      uint32_t pr = 0, acc_it = 0, bs = 0, ds = 0;  // pair, its token slot pair (pr % 3) and DONE (pr % 6)
       bool ok = true;
       bool ready = false;  // the next pair's barrier was already seen complete
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++acc_it) {
@@ -359,25 +381,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(ACC_EMPTY(b), aph ^ 1u, abort_flag, args.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * kAccCols;
-        const uint32_t n_mma = static_cast<uint32_t>((t.count + 15) & ~15);
-        const uint32_t idesc = umma_idesc_f16_m128(n_mma);
+        const uint32_t idesc = umma_idesc_f16_m128(static_cast<uint32_t>((t.count + 15) & ~15));
         for (int kb = 0; kb < nk; kb += 2, ++pr) {
-          const uint32_t ps = pr & 1u, ph = (pr >> 1) & 1u;
-          if (!ready && !mbar_wait(FULL(ps), ph, abort_flag, args.status)) { ok = false; break; }
+          const uint32_t ps = pr & 1u;
+          if (!ready && !mbar_wait(FULL(ps), (pr >> 1) & 1u, abort_flag, args.status)) { ok = false; break; }
           tc_fence_after();
           // look at the next pair's barrier now, while this pair's MMAs queue up
           ready = mbar_try_wait(FULL(ps ^ 1u), ((pr + 1) >> 1) & 1u);
-          const int nst = min(2, nk - kb);
-          for (int h = 0; h < nst; ++h) {
-            const uint32_t a_tmem = tmem_base + kACol0 + (2 * ps + h) * kAStageCols;
-            const uint64_t bdesc = umma_desc_sw128(sbase + CF::kBOff + (2 * ps + h) * kBBytes);
-#pragma unroll
-            for (int k = 0; k < BK / 16; ++k) {
-              // K = 16 per MMA: +8 TMEM columns of A, +32 bytes (+2 in the start field) of B
-              umma_f16_ts(d_tmem, a_tmem + 8u * k, bdesc + 2u * k, idesc, (kb | h | k) != 0 ? 1u : 0u);
-            }
+          const uint32_t a = a_base + ps * (2 * kAStageCols);
+          const uint64_t bd = b_base + bs * (2 * kBStep);
+          // K = 16 per MMA: +8 TMEM columns of A, +32 bytes (+2 in the start field) of B
+          umma_f16_ts(d_tmem, a, bd, idesc, kb != 0 ? 1u : 0u);
+          umma_f16_ts(d_tmem, a + 8u, bd + 2u, idesc, 1u);
+          umma_f16_ts(d_tmem, a + 16u, bd + 4u, idesc, 1u);
+          umma_f16_ts(d_tmem, a + 24u, bd + 6u, idesc, 1u);
+          if (kb + 1 < nk) {
+            umma_f16_ts(d_tmem, a + kAStageCols, bd + kBStep, idesc, 1u);
+            umma_f16_ts(d_tmem, a + kAStageCols + 8u, bd + kBStep + 2u, idesc, 1u);
+            umma_f16_ts(d_tmem, a + kAStageCols + 16u, bd + kBStep + 4u, idesc, 1u);
+            umma_f16_ts(d_tmem, a + kAStageCols + 24u, bd + kBStep + 6u, idesc, 1u);
           }
-          umma_commit(EMPTY(ps));
+          umma_commit(DONE(ds));
+          if (++bs == static_cast<uint32_t>(kBPairs)) bs = 0;
+          if (++ds == static_cast<uint32_t>(kDonePairs)) ds = 0;
         }
         if (!ok) break;
         umma_commit(ACC_FULL(b));
@@ -452,6 +478,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         } else {
+          // w = fp16(level) * fp16(absmax), rounded to fp16 (an absmax beyond the fp16 range
+          // is reported and clamped)
+          if (!(a <= 65504.0f)) {
+            report(args.status, MOEQ_ERR_RANGE);
+            a = 65504.0f;
+          }
+          const __half2 a2 = __float2half2_rn(a);
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
             const uint32_t wv[4] = {cw[q].x, cw[q].y, cw[q].z, cw[q].w};
@@ -459,18 +492,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 4; ++j) {
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
-                // byte k of the word holds elements 2k (high nibble) and 2k+1
-                const uint32_t addr = __byte_perm(wv[j], lane8, 0x5504u | (static_cast<uint32_t>(k) << 4));
-                const float2 c = *reinterpret_cast<const float2 *>(smem + CF::kLutOff + addr);
-                const float2 w = fmul2(c, a);
-                o[16 * q + 4 * j + k] = pack_f16(w.x, w.y);
+                // byte k of the word holds elements 2k (high nibble) and 2k+1; its entry is at
+                // byte*128 + lane*4 = ((byte << 8) | lane*8) >> 1
+                const uint32_t addr = __byte_perm(wv[j], lane8, 0x5504u | (static_cast<uint32_t>(k) << 4)) >> 1;
+                const __half2 c = *reinterpret_cast<const __half2 *>(smem + CF::kLutOff + addr);
+                const __half2 w = __hmul2(c, a2);
+                o[16 * q + 4 * j + k] = *reinterpret_cast<const uint32_t *>(&w);
               }
             }
           }
         }
-        // this stage's A slot: half (kb & 1) of the pair's slot
-        const uint32_t pr = pr0 + (kb >> 1), ps = pr & 1u, ph = (pr >> 1) & 1u;
-        if (!mbar_wait(EMPTY(ps), ph ^ 1u, abort_flag, args.status)) { ok = false; break; }
+        // this stage's A slot: half (kb & 1) of slot pr % 2, last read by the MMAs of pair pr - 2
+        const uint32_t pr = pr0 + (kb >> 1), ps = pr & 1u;
+        if (pr >= 2) {
+          const uint32_t j = pr - 2;
+          if (!mbar_wait(DONE(j % kDonePairs), (j / kDonePairs) & 1u, abort_flag, args.status)) { ok = false; break; }
+        }
         tc_fence_after();
         const uint32_t tcol = trow + (2 * ps + (kb & 1)) * kAStageCols;
         tmem_st_32x32b_x16(tcol, *reinterpret_cast<const uint32_t(*)[16]>(o));
