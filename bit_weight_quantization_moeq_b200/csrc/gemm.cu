@@ -20,13 +20,15 @@
 //               warp w reads TMEM lanes 32*(w%4).. and half the tile's columns
 //   warps 8-23  dequant: packed codes (TMA'd into SMEM) -> fp16 A stage in TMEM, one
 //               weight row per thread; four groups of 4 warps take K stages in turn
-//   warp 24     producer: TMA of the token tile (B, 128B swizzle) and of the code tiles
-//   warp 25     TMEM allocation and the single-thread tcgen05.mma issue
+//   warp 24     TMA of the packed-code tiles
+//   warp 25     TMA of the token tiles, a pair of K stages at a time
+//   warp 26     TMEM allocation and the single-thread tcgen05.mma issue (8 MMAs per pair)
+//   warp 27     relay: a pair's token tiles have landed -> the pair's full barrier
 // TMEM (512 columns): two 192-column fp32 accumulators (the epilogue of one tile overlaps
-// the mainloop of the next) and a 4-deep ring of 32-column fp16 A stages.  The CTA is persistent over a tile list
-// derived on the device from the routing (per-expert token counts).
-// Every mbarrier wait is bounded (2 s); a timeout raises MOEQ_ERR_TIMEOUT and the CTA
-// drains its in-flight copies and MMAs, frees TMEM and returns.
+// the mainloop of the next) and 4 32-column fp16 A stages (2 pairs).  The CTA is
+// persistent over a tile list derived on the device from the routing (per-expert token
+// counts).  Every mbarrier wait is bounded (2 s); a timeout raises MOEQ_ERR_TIMEOUT and
+// the CTA drains its in-flight copies and MMAs, frees TMEM and returns.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>

@@ -38,13 +38,14 @@ __constant__ float kNF4[16] = {
 // 0.08 apart), so with base[m] = #{j : cell(t_j) < m} and thr[m] the threshold in
 // cell m (+inf if none), monotonicity gives exactly
 //   code(n) = base[cell(n)] + (n > thr[cell(n)]).
-// The two 32-entry tables live in shared memory (one bank per entry: no conflicts).
+// The two tables live in shared memory as one 32-entry array of (thr, base) pairs: one
+// 8-byte load per element.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int nf4_cell(float n) {
   return __float_as_int(__fmaf_rn(n, 15.0f, 12582927.0f)) & 31;
 }
 
-__device__ void build_nf4_cells(float *thr, int *base) {
+__device__ void build_nf4_cells(uint2 *cells) {
   const int m = threadIdx.x;
   if (m < 32) {
     int b = 0;
@@ -56,9 +57,14 @@ __device__ void build_nf4_cells(float *thr, int *base) {
       if (cj < m) ++b;
       else if (cj == m) th = t;
     }
-    thr[m] = th;
-    base[m] = b;
+    cells[m] = make_uint2(__float_as_uint(th), static_cast<uint32_t>(b));
   }
+}
+
+// (acc << 4) + code(n), n in cell c: appends the 4-bit code of n below the codes in acc
+__device__ __forceinline__ uint32_t nf4_push(uint32_t acc, float n, int c, const uint2 *cells) {
+  const uint2 tb = cells[c];
+  return (acc << 4) + tb.y + (n > __uint_as_float(tb.x) ? 1u : 0u);
 }
 
 // fl(x / a) for |x| <= a, a a normal fp32 number >= 2^-120, r = RN(1/a):
@@ -113,8 +119,7 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4 v, float (&f)[8]) {
 // 4 lanes per block, absmax by two xor-shuffles inside the 4-lane group.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void nf4_quarter(const uint4 v0, const uint4 v1, size_t q, uint32_t lane,
-                                            const float *thr, const int *base, uint2 *codes,
-                                            float *absmax) {
+                                            const uint2 *cells, uint2 *codes, float *absmax) {
   float x[16];
   {
     float a8[8], b8[8];
@@ -133,50 +138,49 @@ __device__ __forceinline__ void nf4_quarter(const uint4 v0, const uint4 v1, size
   m = fmaxf(m, __shfl_xor_sync(gmask, m, 1, 4));
   m = fmaxf(m, __shfl_xor_sync(gmask, m, 2, 4));
   const float a = m;
-  uint32_t code[16];
+  // word h of the output holds elements 8h..8h+7; byte k of it is (code(2k) << 4) | code(2k+1),
+  // so the codes are pushed in the order 6 7 4 5 2 3 0 1
+  uint32_t out[2] = {0u, 0u};
   if (a == 0.0f || a >= 0x1p-120f) {
     // the division and the cell map two elements at a time (fp32x2)
     const float r = (a == 0.0f) ? 0.0f : __frcp_rn(a);
     const uint64_t r2 = f2u(r, r), na2 = f2u(-a, -a);
     const uint64_t k15 = f2u(15.0f, 15.0f), kc = f2u(12582927.0f, 12582927.0f);
 #pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-      const uint64_t x2 = f2u(x[i], x[i + 1]);
-      const uint64_t q0 = mul2(x2, r2);
-      const uint64_t e = fma2(na2, q0, x2);
-      const uint64_t n2 = fma2(e, r2, q0);
-      const uint64_t f2 = fma2(n2, k15, kc);
-      const int c0 = static_cast<int>(static_cast<uint32_t>(f2) & 31u);
-      const int c1 = static_cast<int>(static_cast<uint32_t>(f2 >> 32) & 31u);
-      code[i] = static_cast<uint32_t>(base[c0] + (lo_f(n2) > thr[c0] ? 1 : 0));
-      code[i + 1] = static_cast<uint32_t>(base[c1] + (hi_f(n2) > thr[c1] ? 1 : 0));
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+      for (int p = 3; p >= 0; --p) {
+        const int i = 8 * h + 2 * p;
+        const uint64_t x2 = f2u(x[i], x[i + 1]);
+        const uint64_t q0 = mul2(x2, r2);
+        const uint64_t e = fma2(na2, q0, x2);
+        const uint64_t n2 = fma2(e, r2, q0);
+        const uint64_t f2 = fma2(n2, k15, kc);
+        out[h] = nf4_push(out[h], lo_f(n2), static_cast<int>(static_cast<uint32_t>(f2) & 31u), cells);
+        out[h] = nf4_push(out[h], hi_f(n2), static_cast<int>(static_cast<uint32_t>(f2 >> 32) & 31u), cells);
+      }
     }
   } else {  // tiny (subnormal-range) absmax: plain IEEE divide
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float n = __fdiv_rn(x[i], a);
-      const int c = nf4_cell(n);
-      code[i] = static_cast<uint32_t>(base[c] + (n > thr[c] ? 1 : 0));
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+      for (int p = 3; p >= 0; --p) {
+        const int i = 8 * h + 2 * p;
+        const float n0 = __fdiv_rn(x[i], a), n1 = __fdiv_rn(x[i + 1], a);
+        out[h] = nf4_push(out[h], n0, nf4_cell(n0), cells);
+        out[h] = nf4_push(out[h], n1, nf4_cell(n1), cells);
+      }
     }
   }
-  uint2 out;
-  out.x = 0;
-  out.y = 0;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    out.x |= ((code[2 * k] << 4) | code[2 * k + 1]) << (8 * k);
-    out.y |= ((code[8 + 2 * k] << 4) | code[8 + 2 * k + 1]) << (8 * k);
-  }
-  codes[q] = out;
+  codes[q] = make_uint2(out[0], out[1]);
   if ((lane & 3u) == 0) absmax[q >> 2] = a;
 }
 
 __global__ void __launch_bounds__(256) k_quant_nf4(const uint4 *__restrict__ w,
                                                    uint2 *__restrict__ codes,
                                                    float *__restrict__ absmax, size_t nquarters) {
-  __shared__ float thr[32];
-  __shared__ int base[32];
-  build_nf4_cells(thr, base);
+  __shared__ uint2 cells[32];
+  build_nf4_cells(cells);
   __syncthreads();
   const uint32_t lane = threadIdx.x & 31u;
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
@@ -185,12 +189,12 @@ __global__ void __launch_bounds__(256) k_quant_nf4(const uint4 *__restrict__ w,
   for (; q + stride < nquarters; q += 2 * stride) {
     const uint4 a0 = ld_stream_u4(w + 2 * q), a1 = ld_stream_u4(w + 2 * q + 1);
     const uint4 b0 = ld_stream_u4(w + 2 * (q + stride)), b1 = ld_stream_u4(w + 2 * (q + stride) + 1);
-    nf4_quarter(a0, a1, q, lane, thr, base, codes, absmax);
-    nf4_quarter(b0, b1, q + stride, lane, thr, base, codes, absmax);
+    nf4_quarter(a0, a1, q, lane, cells, codes, absmax);
+    nf4_quarter(b0, b1, q + stride, lane, cells, codes, absmax);
   }
   if (q < nquarters) {
     const uint4 a0 = ld_stream_u4(w + 2 * q), a1 = ld_stream_u4(w + 2 * q + 1);
-    nf4_quarter(a0, a1, q, lane, thr, base, codes, absmax);
+    nf4_quarter(a0, a1, q, lane, cells, codes, absmax);
   }
 }
 
