@@ -226,12 +226,22 @@ __global__ void __launch_bounds__(256) k_dq_chunk_sum(const float *__restrict__ 
   }
 }
 
+// The chunk sums of expert e added in chunk order; their loads are issued eight at a time
+// (the additions stay in order, so the result is the sequential sum).
 __global__ void k_dq_offset(const double *__restrict__ S, int E, int nb, int nblk,
                             float *__restrict__ off) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= E) return;
+  const double *src = S + static_cast<size_t>(e) * nblk;
   double t = 0.0;
-  for (int c = 0; c < nblk; ++c) t = __dadd_rn(t, S[static_cast<size_t>(e) * nblk + c]);
+  for (int c0 = 0; c0 < nblk; c0 += 8) {
+    double v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = (c0 + j < nblk) ? src[c0 + j] : 0.0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (c0 + j < nblk) t = __dadd_rn(t, v[j]);
+  }
   off[e] = __double2float_rn(__ddiv_rn(t, static_cast<double>(nb)));
 }
 

@@ -43,12 +43,14 @@ __global__ void __launch_bounds__(256) k_route_count(const IdxT *__restrict__ id
   if (chunk >= nchunks) return;  // whole warp; no block-wide barrier below
   int32_t *h = hist + warp * E;
   for (int e = lane; e < E; e += 32) h[e] = 0;
+  // all of the warp's index loads first, then the histogram updates
+  int ev[kSteps];
+#pragma unroll
+  for (int st = 0; st < kSteps; ++st) ev[st] = load_expert(idx, chunk * kRouteChunk + st * 32 + lane, S, E, status);
   __syncwarp();
-  for (int st = 0; st < kSteps; ++st) {
-    const int p = chunk * kRouteChunk + st * 32 + lane;
-    const int e = load_expert(idx, p, S, E, status);
-    if (e >= 0) atomicAdd(&h[e], 1);
-  }
+#pragma unroll
+  for (int st = 0; st < kSteps; ++st)
+    if (ev[st] >= 0) atomicAdd(&h[ev[st]], 1);
   __syncwarp();
   int32_t *dst = counts_chunk + static_cast<size_t>(chunk) * E;
   for (int e = lane; e < E; e += 32) dst[e] = h[e];
@@ -94,11 +96,16 @@ __global__ void __launch_bounds__(1024) k_route_scan(const int32_t *__restrict__
   const int e = threadIdx.x;
   int tot = 0;
   if (e < E) {
-    for (int c = 0; c < nchunks; ++c) {
-      const size_t at = static_cast<size_t>(c) * E + e;
-      const int v = counts_chunk[at];
-      chunk_base[at] = tot;
-      tot += v;
+    // eight chunks' counts in flight at a time
+    for (int c0 = 0; c0 < nchunks; c0 += 8) {
+      int v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = (c0 + j < nchunks) ? counts_chunk[static_cast<size_t>(c0 + j) * E + e] : 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (c0 + j < nchunks) chunk_base[static_cast<size_t>(c0 + j) * E + e] = tot;
+        tot += v[j];
+      }
     }
   }
   const int off = block_exclusive_scan(tot, warp_tot, &total_cnt);
@@ -131,9 +138,13 @@ __global__ void __launch_bounds__(256) k_route_scatter(const IdxT *__restrict__ 
   for (int e = lane; e < E; e += 32) running[e] = base[e];
   __syncwarp();
   const unsigned lt = (1u << lane) - 1u;
+  int ev[kSteps];
+#pragma unroll
+  for (int st = 0; st < kSteps; ++st) ev[st] = load_expert(idx, chunk * kRouteChunk + st * 32 + lane, S, E, nullptr);
+#pragma unroll
   for (int st = 0; st < kSteps; ++st) {
     const int p = chunk * kRouteChunk + st * 32 + lane;
-    const int e = load_expert(idx, p, S, E, nullptr);
+    const int e = ev[st];
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     if (e >= 0) {
       const int rank = __popc(peers & lt);
@@ -145,10 +156,100 @@ __global__ void __launch_bounds__(256) k_route_scatter(const IdxT *__restrict__ 
   }
 }
 
+// The same three steps in one CTA of 1024 threads, for the small problems where launch
+// latency dominates (a few thousand pairs): the per-chunk table (at most kFusedChunks chunks, each walked in
+// order by one warp) lives in shared memory, so the whole routing is one launch.
+constexpr int kFusedChunks = 128;
+constexpr int kFusedMaxE = 256;
+constexpr int kFusedMaxS = 4096;  // beyond, one SM walking the pairs is slower than three launches
+
+template <typename IdxT>
+__global__ void __launch_bounds__(1024) k_route_fused(const IdxT *__restrict__ idx, int S, int E,
+                                                     int nchunks, int chunk, int32_t *__restrict__ counts,
+                                                     int32_t *__restrict__ offsets,
+                                                     int32_t *__restrict__ ntile_prefix,
+                                                     int32_t *__restrict__ perm, int32_t *status) {
+  extern __shared__ int32_t cc[];  // [nchunks][E]: histograms, then running bases
+  __shared__ int warp_tot[32];
+  __shared__ int total_cnt, total_tiles;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < nchunks * E; i += blockDim.x) cc[i] = 0;
+  __syncthreads();
+  // 1: per-chunk histograms
+  for (int c = warp; c < nchunks; c += 32) {
+    int32_t *h = cc + c * E;
+    const int end = min(S, (c + 1) * chunk);
+    for (int p0 = c * chunk; p0 < end; p0 += 32) {
+      const int p = p0 + lane;
+      const int e = p < end ? load_expert(idx, p, S, E, status) : -1;
+      if (e >= 0) atomicAdd(&h[e], 1);
+    }
+  }
+  __syncthreads();
+  // 2: per expert, the chunks' bases in chunk order; offsets and the token-tile prefix
+  const int e = threadIdx.x;
+  int tot = 0;
+  if (e < E) {
+    for (int c = 0; c < nchunks; ++c) {
+      const int v = cc[c * E + e];
+      cc[c * E + e] = tot;
+      tot += v;
+    }
+  }
+  const int off = block_exclusive_scan(tot, warp_tot, &total_cnt);
+  const int nt = (tot + kTileN - 1) / kTileN;
+  const int ntp = block_exclusive_scan(nt, warp_tot, &total_tiles);
+  if (e < E) {
+    offsets[e] = off;
+    ntile_prefix[e] = ntp;
+    if (counts) counts[e] = tot;
+    for (int c = 0; c < nchunks; ++c) cc[c * E + e] += off;
+  }
+  if (e == 0) {
+    offsets[E] = total_cnt;
+    ntile_prefix[E] = total_tiles;
+  }
+  __syncthreads();
+  // 3: stable scatter, each chunk walked in order by the warp that counted it
+  const unsigned lt = (1u << lane) - 1u;
+  for (int c = warp; c < nchunks; c += 32) {
+    int32_t *running = cc + c * E;
+    const int end = min(S, (c + 1) * chunk);
+    for (int p0 = c * chunk; p0 < end; p0 += 32) {
+      const int p = p0 + lane;
+      const int ex = p < end ? load_expert(idx, p, S, E, nullptr) : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, ex);
+      if (ex >= 0) perm[running[ex] + __popc(peers & lt)] = p;
+      __syncwarp();
+      if (ex >= 0 && (peers & lt) == 0) running[ex] += __popc(peers);
+      __syncwarp();
+    }
+  }
+}
+
 cudaError_t launch_route(const void *idx, bool idx64, int S, int E, int nchunks,
                          int32_t *counts_chunk, int32_t *chunk_base, int32_t *counts,
                          int32_t *offsets, int32_t *ntile_prefix, int32_t *perm, int32_t *status,
                          cudaStream_t s, int *launches) {
+  if (S <= kFusedMaxS && E <= kFusedMaxE) {
+    // chunks of a multiple of 32 pairs, at most kFusedChunks of them
+    const int per = (S + kFusedChunks - 1) / kFusedChunks;
+    const int chunk = ((per + 31) / 32) * 32 > 32 ? ((per + 31) / 32) * 32 : 32;
+    const int nfc = (S + chunk - 1) / chunk;
+    const size_t shm = static_cast<size_t>(nfc) * E * sizeof(int32_t);
+    static bool attr = false;
+    if (!attr) {
+      const int mx = kFusedChunks * kFusedMaxE * static_cast<int>(sizeof(int32_t));
+      if (cudaFuncSetAttribute(k_route_fused<long long>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx) != cudaSuccess ||
+          cudaFuncSetAttribute(k_route_fused<int32_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx) != cudaSuccess)
+        return cudaGetLastError();
+      attr = true;
+    }
+    if (idx64) k_route_fused<long long><<<1, 1024, shm, s>>>(static_cast<const long long *>(idx), S, E, nfc, chunk, counts, offsets, ntile_prefix, perm, status);
+    else k_route_fused<int32_t><<<1, 1024, shm, s>>>(static_cast<const int32_t *>(idx), S, E, nfc, chunk, counts, offsets, ntile_prefix, perm, status);
+    *launches += 1;
+    return cudaGetLastError();
+  }
   const int blocks = (nchunks + kWarpsPerBlock - 1) / kWarpsPerBlock;
   const size_t shm = static_cast<size_t>(kWarpsPerBlock) * E * sizeof(int32_t);
   if (idx64) k_route_count<long long><<<blocks, 256, shm, s>>>(static_cast<const long long *>(idx), S, E, nchunks, counts_chunk, status);

@@ -52,7 +52,10 @@ def run_forward(inp, mode, **kw):
 # ---------------------------------------------------------------------------
 # routing
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("T,K,E", [(1, 1, 8), (7, 2, 8), (300, 8, 64), (5000, 8, 128), (4096, 2, 1000)])
+# (single-launch routing up to 4096 pairs and 256 experts, the first three cases; the
+# chunked three-kernel path beyond)
+@pytest.mark.parametrize("T,K,E", [(1, 1, 8), (7, 2, 8), (300, 8, 64), (5000, 8, 128), (32768, 8, 256),
+                                   (4096, 2, 1000), (40000, 8, 64), (33000, 8, 256)])
 @pytest.mark.parametrize("dtype", [torch.int32, torch.int64])
 def test_route_parity(T, K, E, dtype):
     g = torch.Generator().manual_seed(T * 31 + E)

@@ -39,8 +39,11 @@ def _noalloc(f, idx, E, status):
 def test_route_noalloc_matches_route_on_two_calls_in_a_row():
     m, f = _lib()
     g = torch.Generator().manual_seed(5)
-    cases = [(4096, 8, 64, torch.int32),      # 64 chunks x 64 experts of scratch
-             (777, 2, 128, torch.int64)]      # fewer chunks, more experts: a different layout
+    # routing problems up to 4096 pairs and 256 experts take a single launch that keeps its
+    # tables in shared memory; larger ones go through the scratch array
+    cases = [(40000, 8, 64, torch.int32),     # 625 chunks x 64 experts of scratch
+             (3000, 2, 600, torch.int64),     # fewer chunks, more experts: a different layout
+             (500, 8, 64, torch.int32)]       # the single-launch form
     for T, K, E, dt in cases:
         idx = torch.randint(0, E, (T, K), generator=g).to(dt).cuda()
         status = torch.zeros(1, dtype=torch.int32, device="cuda")
