@@ -105,6 +105,25 @@ __device__ __forceinline__ uint4 ld_stream_u4(const void *p) {
   return v;
 }
 
+// 32 bytes in one 256-bit load (the address must be 32-byte aligned)
+__device__ __forceinline__ void ld_stream_v8(const void *p, uint4 &a, uint4 &b) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+               : "l"(p));
+}
+
+// the 32 bytes of quarter q: one 256-bit load when the source is 32-byte aligned, else two
+// 16-byte loads
+template <bool V8>
+__device__ __forceinline__ void load_quarter(const uint4 *w, size_t q, uint4 &a, uint4 &b) {
+  if (V8) {
+    ld_stream_v8(w + 2 * q, a, b);
+  } else {
+    a = ld_stream_u4(w + 2 * q);
+    b = ld_stream_u4(w + 2 * q + 1);
+  }
+}
+
 __device__ __forceinline__ void unpack_bf16x8(const uint4 v, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -176,6 +195,7 @@ __device__ __forceinline__ void nf4_quarter(const uint4 v0, const uint4 v1, size
   if ((lane & 3u) == 0) absmax[q >> 2] = a;
 }
 
+template <bool V8>
 __global__ void __launch_bounds__(256) k_quant_nf4(const uint4 *__restrict__ w,
                                                    uint2 *__restrict__ codes,
                                                    float *__restrict__ absmax, size_t nquarters) {
@@ -187,13 +207,15 @@ __global__ void __launch_bounds__(256) k_quant_nf4(const uint4 *__restrict__ w,
   size_t q = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   // two quarters in flight per thread
   for (; q + stride < nquarters; q += 2 * stride) {
-    const uint4 a0 = ld_stream_u4(w + 2 * q), a1 = ld_stream_u4(w + 2 * q + 1);
-    const uint4 b0 = ld_stream_u4(w + 2 * (q + stride)), b1 = ld_stream_u4(w + 2 * (q + stride) + 1);
+    uint4 a0, a1, b0, b1;
+    load_quarter<V8>(w, q, a0, a1);
+    load_quarter<V8>(w, q + stride, b0, b1);
     nf4_quarter(a0, a1, q, lane, cells, codes, absmax);
     nf4_quarter(b0, b1, q + stride, lane, cells, codes, absmax);
   }
   if (q < nquarters) {
-    const uint4 a0 = ld_stream_u4(w + 2 * q), a1 = ld_stream_u4(w + 2 * q + 1);
+    uint4 a0, a1;
+    load_quarter<V8>(w, q, a0, a1);
     nf4_quarter(a0, a1, q, lane, cells, codes, absmax);
   }
 }
@@ -462,8 +484,12 @@ cudaError_t launch_quant_nf4(const void *w, size_t n_elems, uint8_t *codes, floa
                              int sm_count, cudaStream_t s, int *launches) {
   const size_t nq = n_elems / 16;
   const int grid = grid_for((nq + 1) / 2, 256, sm_count, 8);
-  k_quant_nf4<<<grid, 256, 0, s>>>(reinterpret_cast<const uint4 *>(w), reinterpret_cast<uint2 *>(codes),
-                                   absmax, nq);
+  if ((reinterpret_cast<uintptr_t>(w) & 31u) == 0)
+    k_quant_nf4<true><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4 *>(w), reinterpret_cast<uint2 *>(codes),
+                                           absmax, nq);
+  else
+    k_quant_nf4<false><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4 *>(w), reinterpret_cast<uint2 *>(codes),
+                                            absmax, nq);
   ++*launches;
   return cudaGetLastError();
 }

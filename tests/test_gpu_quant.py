@@ -74,6 +74,19 @@ def test_quantize_parity_random(mode, shape):
     assert_packed_equal(gpu_packed_numpy(p), oracle_quantize(bits(w), mode), mode)
 
 
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_quantize_source_aligned_to_16_bytes_only(mode):
+    # a source 16 bytes past a 32-byte boundary takes the 16-byte-load path of the NF4
+    # quantizer (32-byte-aligned sources use single 256-bit loads)
+    E, R, C = 3, 17, 192
+    base = rand_w((1, 1, E * R * C + 64), seed=77 + mode, outliers=(mode == 2)).view(-1)
+    w = base[8:8 + E * R * C].view(E, R, C)
+    assert w.data_ptr() % 32 == 16
+    p = quantize(w, mode)
+    torch.cuda.synchronize()
+    assert_packed_equal(gpu_packed_numpy(p), oracle_quantize(bits(w), mode), mode)
+
+
 @pytest.mark.parametrize("mode", [0, 2])
 def test_quantize_parity_every_mantissa_pair(mode):
     w = mantissa_pair_tensor(64).cuda()
