@@ -125,6 +125,19 @@ def test_forward_bad_index_dropped_duplicates_added_and_dtypes():
     assert int(status.item()) == 9
 
 
+def test_forward_hidden_beyond_fp16_saturates_and_reports():
+    # the tensor cores take fp16 tokens: a hidden value beyond +-65504 saturates and raises
+    # MOEQ_ERR_RANGE (11); the other tokens are unaffected
+    T = 40
+    inp = make_inputs(8, 256, 128, T, 2, seed=13)
+    inp["hidden"][3, 5] = 1.0e5
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = run_forward(inp, 0, d_status=status)
+    assert int(status.item()) == 11
+    others = [t for t in range(T) if t != 3]
+    check_forward(out, oracle_forward(inp, 0, tokens=others), tokens=others)
+
+
 def test_forward_top_all_experts_uniform():
     E, H, I, T = 8, 256, 128, 33
     inp = make_inputs(E, H, I, T, E, seed=21)
