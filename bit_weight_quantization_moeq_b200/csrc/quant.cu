@@ -223,48 +223,65 @@ __global__ void __launch_bounds__(256) k_quant_nf4(const uint4 *__restrict__ w,
 // ---------------------------------------------------------------------------
 // a2: double quantization of absmax [E, nb] (fixed-order fp64 mean, int8 blocks of 256)
 // ---------------------------------------------------------------------------
-// Chunk sums: 8 chunks of 256 per block, staged in shared memory, each summed
+// Chunk sums: kDqSumChunks chunks of 256 per block, staged in shared memory (coalesced
+// loads, row pitch 257 so that the summing threads hit distinct banks), each summed
 // sequentially by one thread (the order is part of the definition).
+constexpr int kDqSumChunks = 64;
 __global__ void __launch_bounds__(256) k_dq_chunk_sum(const float *__restrict__ absmax, int nb,
                                                       int nblk, int nchunks_total,
                                                       double *__restrict__ S) {
-  __shared__ float buf[8][257];
-  const int c0 = blockIdx.x * 8;
-  for (int j = 0; j < 8; ++j) {
-    const int g = c0 + j;
-    if (g >= nchunks_total) break;
-    const int e = g / nblk, c = g - e * nblk;
-    const int i = c * 256 + static_cast<int>(threadIdx.x);
-    buf[j][threadIdx.x] = (i < nb) ? absmax[static_cast<size_t>(e) * nb + i] : 0.0f;
+  extern __shared__ float buf[];  // [kDqSumChunks][257]
+  const int c0 = blockIdx.x * kDqSumChunks;
+  // thread t stages element t of every chunk (256 threads = one chunk row), 16 chunks' loads
+  // in flight before their shared-memory stores
+  const int i = threadIdx.x;
+  for (int j0 = 0; j0 < kDqSumChunks; j0 += 16) {
+    float v[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int g = c0 + j0 + u;
+      v[u] = 0.0f;
+      if (g < nchunks_total) {
+        const int e = g / nblk, c = g - e * nblk;
+        const int at = c * 256 + i;
+        if (at < nb) v[u] = absmax[static_cast<size_t>(e) * nb + at];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) buf[(j0 + u) * 257 + i] = v[u];
   }
   __syncthreads();
-  if (threadIdx.x < 8) {
+  if (threadIdx.x < kDqSumChunks) {
     const int g = c0 + threadIdx.x;
     if (g < nchunks_total) {
       double s = 0.0;
-      for (int i = 0; i < 256; ++i) s = __dadd_rn(s, static_cast<double>(buf[threadIdx.x][i]));
+      for (int i = 0; i < 256; ++i) s = __dadd_rn(s, static_cast<double>(buf[threadIdx.x * 257 + i]));
       S[g] = s;
     }
   }
 }
 
-// The chunk sums of expert e added in chunk order; their loads are issued eight at a time
-// (the additions stay in order, so the result is the sequential sum).
-__global__ void k_dq_offset(const double *__restrict__ S, int E, int nb, int nblk,
-                            float *__restrict__ off) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= E) return;
+// One warp per expert: the lanes stage the expert's chunk sums in shared memory (coalesced,
+// all loads in flight together), then lane 0 adds them in chunk order (the sequential sum).
+constexpr int kDqOffWarps = 8;
+constexpr int kDqOffMaxChunks = 512;   // chunk sums staged per pass (8 warps x 4 KB)
+__global__ void __launch_bounds__(kDqOffWarps * 32) k_dq_offset(const double *__restrict__ S, int E, int nb,
+                                                                int nblk, float *__restrict__ off) {
+  __shared__ double buf[kDqOffWarps][kDqOffMaxChunks];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * kDqOffWarps + warp;
+  if (e >= E) return;  // whole warp; no block-wide barrier below
   const double *src = S + static_cast<size_t>(e) * nblk;
   double t = 0.0;
-  for (int c0 = 0; c0 < nblk; c0 += 8) {
-    double v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = (c0 + j < nblk) ? src[c0 + j] : 0.0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (c0 + j < nblk) t = __dadd_rn(t, v[j]);
+  for (int c0 = 0; c0 < nblk; c0 += kDqOffMaxChunks) {
+    const int n = min(kDqOffMaxChunks, nblk - c0);
+    for (int c = lane; c < n; c += 32) buf[warp][c] = src[c0 + c];
+    __syncwarp();
+    if (lane == 0)
+      for (int c = 0; c < n; ++c) t = __dadd_rn(t, buf[warp][c]);
+    __syncwarp();
   }
-  off[e] = __double2float_rn(__ddiv_rn(t, static_cast<double>(nb)));
+  if (lane == 0) off[e] = __double2float_rn(__ddiv_rn(t, static_cast<double>(nb)));
 }
 
 // One warp per 256-block: v = fl(a - off), s = max|v|, q = rint(fl(fl(127 v) / s)).
@@ -499,8 +516,17 @@ cudaError_t launch_double_quant(const float *absmax_f32, int E, int nb, double *
                                 int *launches) {
   const int nblk = (nb + 255) / 256;
   const int total = E * nblk;
-  k_dq_chunk_sum<<<(total + 7) / 8, 256, 0, s>>>(absmax_f32, nb, nblk, total, chunk_sums);
-  k_dq_offset<<<(E + 127) / 128, 128, 0, s>>>(chunk_sums, E, nb, nblk, off);
+  const size_t sum_smem = static_cast<size_t>(kDqSumChunks) * 257 * sizeof(float);
+  static bool sum_attr = false;
+  if (!sum_attr) {
+    const cudaError_t e = cudaFuncSetAttribute(k_dq_chunk_sum, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(sum_smem));
+    if (e != cudaSuccess) return e;
+    sum_attr = true;
+  }
+  k_dq_chunk_sum<<<(total + kDqSumChunks - 1) / kDqSumChunks, 256, sum_smem, s>>>(absmax_f32, nb, nblk, total,
+                                                                                  chunk_sums);
+  k_dq_offset<<<(E + kDqOffWarps - 1) / kDqOffWarps, kDqOffWarps * 32, 0, s>>>(chunk_sums, E, nb, nblk, off);
   k_dq_quant<<<(total + 7) / 8, 256, 0, s>>>(absmax_f32, off, E, nb, nblk, q_out, scale);
   *launches += 3;
   return cudaGetLastError();

@@ -106,6 +106,15 @@ def test_double_quant_partial_blocks_and_constant_expert():
     assert np.all(ref["absmax_q"][1] == 0)
 
 
+def test_double_quant_offset_over_many_chunks():
+    # one expert with 1040 chunks of 256 absmax values: the per-expert offset is summed in
+    # several staged passes and must still equal the oracle's sequential sum
+    w = rand_w((1, 4096, 4160), seed=29)
+    p = quantize(w, 1)
+    torch.cuda.synchronize()
+    assert_packed_equal(gpu_packed_numpy(p), oracle_quantize(bits(w), 1), 1)
+
+
 @pytest.mark.parametrize("mode", [0, 1, 2])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 def test_dequantize_parity(mode, out_dtype):
