@@ -32,11 +32,14 @@
  *   of gate_up, never inferred from the shape):
  *     out[t] = sum_k w[t,k] * down_e( silu(gate_e x_t) * up_e x_t ),  e = idx[t,k],
  *   with silu(z) = z / (1 + exp(-z)), fp32 accumulation, the k terms added in k
- *   order, the result rounded once to bf16.  top_k_weights are used as given.  The
- *   tensor-core operands are fp16 (the compute dtype of the pages' bitsandbytes
- *   reproduction, bnb_4bit_compute_dtype=float16): the dequantized weights, the
- *   hidden rows (converted from bf16, exact for 6.1e-5 <= |x| <= 65504) and the
- *   intermediate h; larger magnitudes saturate and report MOEQ_ERR_RANGE.
+ *   order, the result rounded once to bf16 (or returned in fp32, out_dtype MOEQ_F32).
+ *   top_k_weights are used as given.  The tensor-core operands are fp16 (the compute
+ *   dtype of the pages' bitsandbytes reproduction, bnb_4bit_compute_dtype=float16):
+ *   the hidden rows (converted from bf16, exact for 6.1e-5 <= |x| <= 65504), the
+ *   intermediate h, and the weights decoded in the GEMM: fp16(fp16(level) *
+ *   fp16(absmax)) for NF4, the exact code q for int8 (its row scale is applied to the
+ *   fp32 accumulator).  Larger magnitudes saturate and report MOEQ_ERR_RANGE.
+ *   moeq_dequantize is unaffected: it returns the exact dequantized values above.
  *
  * Conventions (every entry point):
  *   - Memory: every pointer argument is a DEVICE pointer, 16-byte aligned, unless the
@@ -79,8 +82,9 @@ typedef enum {
   MOEQ_ERR_TIMEOUT = 8,    /* device: a pipeline wait ran past its limit (a bug) */
   MOEQ_ERR_INDEX = 9,      /* device: a top_k_index value outside [0, E) was dropped */
   MOEQ_ERR_DEVICE = 10,    /* the current device is not compute capability 10.0 */
-  MOEQ_ERR_RANGE = 11      /* device: an activation (hidden or h) beyond the fp16 range of
-                              the tensor-core operands (|v| > 65504) was saturated */
+  MOEQ_ERR_RANGE = 11      /* device: an activation (hidden or h) or an NF4 block absmax
+                              beyond the fp16 range of the tensor-core operands
+                              (|v| > 65504) was saturated */
 } moeq_status;
 
 typedef enum { MOEQ_NF4 = 0, MOEQ_NF4_DQ = 1, MOEQ_INT8_ROW = 2 } moeq_mode;

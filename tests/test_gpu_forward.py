@@ -138,6 +138,16 @@ def test_forward_hidden_beyond_fp16_saturates_and_reports():
     check_forward(out, oracle_forward(inp, 0, tokens=others), tokens=others)
 
 
+def test_forward_nf4_absmax_beyond_fp16_reports():
+    # an NF4 block whose absmax exceeds the fp16 range cannot be an fp16 tensor-core operand:
+    # the GEMM clamps its scale and reports MOEQ_ERR_RANGE (11)
+    inp = make_inputs(8, 256, 128, 64, 2, seed=17)
+    inp["gate_up"][int(inp["top_k_index"][0, 0]), 5, 9] = 1.0e5
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    run_forward(inp, 0, d_status=status)
+    assert int(status.item()) == 11
+
+
 def test_forward_top_all_experts_uniform():
     E, H, I, T = 8, 256, 128, 33
     inp = make_inputs(E, H, I, T, E, seed=21)
